@@ -1,0 +1,66 @@
+"""ctypes loader for the in-tree libwmtp.so (the C ABI declared in include/wmtp.h).
+
+The library must exist: there is no fallback.  Loading raises when it is missing.
+"""
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libwmtp.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "wmtp.h")
+
+STATUS = {
+    0: "WMTP_OK", -1: "WMTP_ERR_ARG", -2: "WMTP_ERR_SHAPE", -3: "WMTP_ERR_ALIGN",
+    -4: "WMTP_ERR_WORKSPACE", -5: "WMTP_ERR_CUDA", -6: "WMTP_ERR_DEVICE_INDEX",
+    -7: "WMTP_ERR_UNSUPPORTED", -8: "WMTP_ERR_TIMEOUT",
+}
+
+
+class WmtpError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+_lib = None
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+F = ctypes.c_float
+SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "wmtp_status_string": ([I], ctypes.c_char_p),
+    "wmtp_workspace_bytes": ([I, I, I, I, I], SZ),
+    "ring_kv_append": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
+    "draft_attn_window": ([P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, SZ, P], I),
+    "draft_attn_full": ([P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, SZ, P], I),
+    "verify_attn": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, SZ, P], I),
+    "accept_greedy": ([P, P, P, I, I, I, P, P, P], I),
+    "wmtp_device_status": ([P], I),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises FileNotFoundError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FileNotFoundError(
+                f"{LIB_PATH} is missing: build it with `python -m long_context_speculative_kv_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            f = getattr(l, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().wmtp_status_string(int(status)).decode()
+
+
+def check(fn: str, status: int) -> None:
+    if status != 0:
+        raise WmtpError(fn, status)

@@ -1,0 +1,142 @@
+"""Python binding of libwmtp.so with the C ABI's names: argument marshalling only.
+
+Tensors are torch CUDA tensors (bf16 for Q/K/V/out, fp32 for logits and LSE, int32/int64 for
+lengths, tables and tokens).  Every call launches the library's kernels on the current torch
+stream (or ``stream``) and returns without synchronizing; errors raise WmtpError.  Shapes:
+
+    q, out        [B, n_q, Hq, 128]        bf16
+    ring_k/v      [B, Hkv, C, 128]         bf16,  ring_len [B] int64
+    k/v pool      [pages, Hkv, 64, 128]    bf16,  page_table [B, max_pages] int32, kv_len [B] int32
+    logits        [B, n_q, V] fp32, tokens / tree_parent / accepted [B, n_q] int32
+"""
+from typing import Optional, Tuple
+
+import torch
+
+from ._lib import check, lib
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _want(t: torch.Tensor, dtype, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != ndim:
+        raise TypeError(f"{name}: expected a {ndim}-d {dtype} tensor")
+    if not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous CUDA tensor")
+
+
+def workspace_bytes(B: int, n_q: int, Hq: int, Hkv: int, D: int = 128) -> int:
+    return int(lib().wmtp_workspace_bytes(B, n_q, Hq, Hkv, D))
+
+
+def alloc_workspace(B: int, n_q: int, Hq: int, Hkv: int, device=None) -> torch.Tensor:
+    n = workspace_bytes(B, n_q, Hq, Hkv)
+    if n == 0:
+        raise ValueError("invalid shape for the workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def ring_kv_append(ring_k, ring_v, ring_len, k_new, v_new, n_sink: int, stream=None) -> None:
+    _want(ring_k, torch.bfloat16, "ring_k", 4)
+    _want(ring_v, torch.bfloat16, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    _want(k_new, torch.bfloat16, "k_new", 4)
+    _want(v_new, torch.bfloat16, "v_new", 4)
+    B, Hkv, C, D = ring_k.shape
+    n_new = k_new.shape[1]
+    if k_new.shape != (B, n_new, Hkv, D) or v_new.shape != k_new.shape or ring_v.shape != ring_k.shape:
+        raise ValueError("ring_kv_append: inconsistent shapes")
+    check("ring_kv_append", lib().ring_kv_append(
+        _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), _ptr(k_new), _ptr(v_new),
+        B, n_new, Hkv, D, int(n_sink), C, _stream(stream)))
+
+
+def _outs(q, out, lse, want_lse):
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def draft_attn_window(q, ring_k, ring_v, ring_len, n_sink: int, window: int, sm_scale: float,
+                      ws: torch.Tensor, out=None, lse=None, want_lse: bool = True,
+                      stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    _want(q, torch.bfloat16, "q", 4)
+    _want(ring_k, torch.bfloat16, "ring_k", 4)
+    _want(ring_v, torch.bfloat16, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    B, n_q, Hq, D = q.shape
+    _, Hkv, C, _ = ring_k.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_window", lib().draft_attn_window(
+        _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), B, n_q, Hq, Hkv, D, int(n_sink),
+        int(window), C, float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def _paged_checks(q, k_pool, v_pool, page_table, kv_len):
+    _want(q, torch.bfloat16, "q", 4)
+    _want(k_pool, torch.bfloat16, "k_pool", 4)
+    _want(v_pool, torch.bfloat16, "v_pool", 4)
+    _want(page_table, torch.int32, "page_table", 2)
+    _want(kv_len, torch.int32, "kv_len", 1)
+    if v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool and v_pool differ in shape")
+
+
+def draft_attn_full(q, k_pool, v_pool, page_table, kv_len, sm_scale: float, ws: torch.Tensor,
+                    out=None, lse=None, want_lse: bool = True, stream=None):
+    _paged_checks(q, k_pool, v_pool, page_table, kv_len)
+    B, n_q, Hq, D = q.shape
+    num_pages, Hkv, P, _ = k_pool.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_full", lib().draft_attn_full(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(kv_len), B, n_q, Hq, Hkv, D, P,
+        page_table.shape[1], num_pages, float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return out, lse
+
+
+def verify_attn(q, k_pool, v_pool, page_table, kv_len, sm_scale: float, ws: torch.Tensor,
+                tree_parent=None, out=None, lse=None, want_lse: bool = True, stream=None):
+    _paged_checks(q, k_pool, v_pool, page_table, kv_len)
+    if tree_parent is not None:
+        _want(tree_parent, torch.int32, "tree_parent", 2)
+    B, n_q, Hq, D = q.shape
+    num_pages, Hkv, P, _ = k_pool.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("verify_attn", lib().verify_attn(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(kv_len), _ptr(tree_parent),
+        B, n_q, Hq, Hkv, D, P, page_table.shape[1], num_pages, float(sm_scale), _ptr(out),
+        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def accept_greedy(logits, tokens, tree_parent=None, accepted=None, n_accepted=None, stream=None):
+    _want(logits, torch.float32, "logits", 3)
+    _want(tokens, torch.int32, "tokens", 2)
+    if tree_parent is not None:
+        _want(tree_parent, torch.int32, "tree_parent", 2)
+    B, n_q, V = logits.shape
+    if accepted is None:
+        accepted = torch.empty((B, n_q), dtype=torch.int32, device=logits.device)
+    if n_accepted is None:
+        n_accepted = torch.empty((B,), dtype=torch.int32, device=logits.device)
+    check("accept_greedy", lib().accept_greedy(
+        _ptr(logits), _ptr(tokens), _ptr(tree_parent), B, n_q, V, _ptr(accepted), _ptr(n_accepted),
+        _stream(stream)))
+    return accepted, n_accepted
+
+
+def device_status(stream=None) -> int:
+    """Reads and clears the device status word (synchronizes the stream); 0 when clean."""
+    return int(lib().wmtp_device_status(_stream(stream)))

@@ -1,0 +1,600 @@
+// attn_kernels.cuh -- split-KV decode/verify attention for sm_100a.
+//
+// One kernel template serves the three attention calls of the Windowed-MTP decode step
+// (Windowed-MTP, arXiv 2607.21535; Pith verdict, pith_extraction.key_machinery):
+//   * draft_attn_window: keys = the attention sink plus the recent window, read from the ring as
+//     at most three contiguous slot ranges (never a dense mask);
+//   * draft_attn_full:   keys = the whole paged KV cache (the native draft it replaces);
+//   * verify_attn:       keys = the paged prefix plus the step's nodes (chain-causal or tree).
+//
+// Work decomposition.  A "unit" is (request b, kv head h, row block rb); its rows are the
+// n_q * G query rows (query i, packed GQA head g: row = i * G + g) of that kv head, 64 per row
+// block.  Its keys are cut into tiles of 64 keys (one page, or a piece of one ring range).  The
+// tiles of all units form one flat sequence of T tiles; CTA c of the P_eff working CTAs takes the
+// tiles [floor(c T / P_eff), floor((c+1) T / P_eff)), so every CTA streams the same number of
+// bytes whatever the lengths and ring wrap (stream-K).  A unit entirely inside one CTA is
+// finished there; otherwise each CTA writes an (o, lse) partial to workspace slot c + u and
+// lse_merge_kernel combines them (slots are unique: c' > c implies u' >= u).
+//
+// Inside a CTA: one producer warp streams K/V tiles with TMA (two 64x64 bf16 boxes per tensor,
+// 128-byte swizzle) through an NSTAGE ring of mbarrier-guarded stages; NMT x NKG consumer warps
+// each own one 16-row m-tile and 64/NKG keys of every tile and run QK^T and PV on the tensor
+// cores (mma.sync m16n8k16 bf16, fp32 accumulate) with an online base-2 softmax.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace wmtp {
+
+constexpr int kD = 128;
+constexpr int kTileKeys = 64;
+constexpr int kRowsPerBlock = 64;
+constexpr int kHalfBytes = kTileKeys * 64 * 2;      // one 64x64 bf16 box: 8 KiB
+constexpr int kTileBytes = 2 * kHalfBytes;          // K or V tile: 16 KiB
+constexpr int kStageBytes = 2 * kTileBytes;         // K + V: 32 KiB
+constexpr int kMaxBatch = 256;
+constexpr float kLn2 = 0.693147180559945309f;
+
+enum SourceKind : int { kSrcPaged = 0, kSrcRing = 1 };
+
+struct AttnArgs {
+    const __nv_bfloat16* q;      // [B, n_q, Hq, D]
+    __nv_bfloat16* out;          // [B, n_q, Hq, D]
+    float* lse;                  // [B, n_q, Hq] or null
+    float* ws_o;                 // [slots][64][D]   normalised partial outputs
+    float* ws_lse;               // [slots][64]      base-2 partial log-sum-exp
+    int B, n_q, Hq, Hkv, G, n_rb;
+    int rows_total;              // n_q * G
+    float scale_log2;            // sm_scale * log2(e)
+    const int* tree_parent;      // [B, n_q] or null (chain / causal)
+    // paged source
+    const int* page_table;       // [B, max_pages]
+    const int* kv_len;           // [B]
+    int max_pages, num_pages;
+    // ring source
+    const long long* ring_len;   // [B]
+    int n_sink, window, capacity;
+    // plan
+    int min_tiles_per_cta;
+};
+
+// Per-stage tile description, written by the producer before the stage's barrier completes.
+struct TileMeta {
+    int b, h, rb, unit;
+    int pos0;       // logical position of the tile's row 0
+    int nvalid;     // rows [0, nvalid) are keys of this unit; 0 = skipped tile
+    int L_tot;      // request length (keys) including this call's n_q positions
+    int flags;      // kFirst | kLast | kWhole
+};
+enum : int { kFirst = 1, kLast = 2, kWhole = 4 };
+
+// ---------------------------------------------------------------------------------------------
+// Key ranges of a request.
+// Ring: sink slots [0, ns) hold positions [0, ns); the recent window positions [r0, L) sit in
+// ring slots starting at slot(r0) and wrap at most once (slot(p) = n_sink + (p - n_sink) mod
+// (C - n_sink)).  Paged: one range of L keys.
+struct Ranges {
+    int n;               // number of ranges (<= 3)
+    int slot0[3], pos0[3], len[3];
+};
+
+__device__ __forceinline__ Ranges ring_ranges(long long L_ll, int s, int W, int C) {
+    Ranges r;
+    r.n = 0;
+    const int L = (int)L_ll;
+    const int ns = L < s ? L : s;
+    if (ns > 0) { r.slot0[r.n] = 0; r.pos0[r.n] = 0; r.len[r.n] = ns; ++r.n; }
+    if (L > s) {
+        const int r0 = (L - W) > s ? (L - W) : s;
+        const int n = L - r0;
+        const int a = s + (r0 - s) % (C - s);
+        const int first = n < (C - a) ? n : (C - a);
+        r.slot0[r.n] = a; r.pos0[r.n] = r0; r.len[r.n] = first; ++r.n;
+        if (n - first > 0) { r.slot0[r.n] = s; r.pos0[r.n] = r0 + first; r.len[r.n] = n - first; ++r.n; }
+    }
+    return r;
+}
+
+template <int SRC>
+__device__ __forceinline__ int request_len(const AttnArgs& a, int b) {
+    long long L = (SRC == kSrcPaged) ? (long long)a.kv_len[b] : a.ring_len[b];
+    if (L < 0) L = 0;
+    if (L > 0x7fffffffll) L = 0x7fffffffll;
+    return (int)L;
+}
+
+template <int SRC>
+__device__ __forceinline__ int request_tiles(const AttnArgs& a, int L) {
+    if (SRC == kSrcPaged) return (L + kTileKeys - 1) / kTileKeys;
+    Ranges r = ring_ranges(L, a.n_sink, a.window, a.capacity);
+    int t = 0;
+    for (int k = 0; k < r.n; ++k) t += (r.len[k] + kTileKeys - 1) / kTileKeys;
+    return t;
+}
+
+__device__ __forceinline__ long long cta_begin(long long c, long long T, long long P) {
+    return c * T / P;
+}
+
+__device__ __forceinline__ int plan_ctas(long long T, int P_launch, int min_tiles) {
+    long long want = (T + min_tiles - 1) / min_tiles;
+    if (want < 1) want = 1;
+    return (int)(want < P_launch ? want : P_launch);
+}
+
+// CTA whose tile range contains tile t (largest c with begin(c) <= t).
+__device__ __forceinline__ int cta_of_tile(long long t, long long T, int P) {
+    long long c = ((t + 1) * P + T - 1) / T - 1;
+    return (int)c;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Shared-memory layout (dynamic; stage buffers 1024-byte aligned for the 128-byte swizzle).
+template <int NMT, int NKG, int NSTAGE>
+struct SmemLayout {
+    static constexpr int kStagesBytes = NSTAGE * kStageBytes;
+    static constexpr int kMergeStride = kD + 4;                      // floats per merge row
+    static constexpr int kMergeFloats = (NKG - 1) * NMT * 16 * kMergeStride;
+    static constexpr int kMergeMLFloats = (NKG - 1) * NMT * 16 * 2;
+    static constexpr int kMergeOff = kStagesBytes;
+    static constexpr int kMergeMLOff = kMergeOff + kMergeFloats * 4;
+    static constexpr int kBarOff = kMergeMLOff + kMergeMLFloats * 4;
+    static constexpr int kMetaOff = kBarOff + (2 * NSTAGE + 1) * 8;
+    static constexpr int kPlanOff = kMetaOff + NSTAGE * (int)sizeof(TileMeta);
+    static constexpr int kPlanBytes = 2 * kMaxBatch * 4;            // tiles per request, length
+    static constexpr int kTotal = kPlanOff + kPlanBytes;
+    static constexpr int kAlloc = kTotal + 1024;                     // slack for base alignment
+};
+
+// Swizzled shared address of 16-byte chunk `chunk` (0..15) of key row `row` in a K/V tile
+// stored as two 64x64 boxes with the TMA 128-byte swizzle (chunk' = chunk ^ (row & 7)).
+__device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t base, int row, int chunk) {
+    return base + (uint32_t)((chunk >> 3) * kHalfBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+// ---------------------------------------------------------------------------------------------
+template <int SRC, int NMT, int NKG, int NSTAGE>
+__global__ void __launch_bounds__((NMT * NKG + 1) * 32, 1)
+attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                  const AttnArgs a) {
+    using L = SmemLayout<NMT, NKG, NSTAGE>;
+    constexpr int NWC = NMT * NKG;            // consumer warps
+    constexpr int KPW = kTileKeys / NKG;      // keys per consumer warp per tile
+    constexpr int NT = KPW / 8;               // S n-tiles per warp
+    static_assert(KPW % 16 == 0, "keys per warp must be a multiple of 16");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* merge_o = reinterpret_cast<float*>(smem + L::kMergeOff);
+    float* merge_ml = reinterpret_cast<float*>(smem + L::kMergeMLOff);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* empty_bar = full_bar + NSTAGE;
+    uint64_t* sync_bar = full_bar + 2 * NSTAGE;   // consumer-warp rendezvous at unit ends
+    TileMeta* meta = reinterpret_cast<TileMeta*>(smem + L::kMetaOff);
+    int* plan_tiles = reinterpret_cast<int*>(smem + L::kPlanOff);
+    int* plan_len = plan_tiles + kMaxBatch;
+    __shared__ long long s_range[2];          // this CTA's [t_begin, t_end)
+    __shared__ int s_peff;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- plan: lengths -> tiles per request -> this CTA's tile range ------------------------
+    if (warp == NWC) {
+        for (int b = lane; b < a.B; b += 32) {
+            const int Lb = request_len<SRC>(a, b);
+            plan_len[b] = Lb;
+            plan_tiles[b] = request_tiles<SRC>(a, Lb);
+        }
+        __syncwarp();
+        if (lane == 0) {
+            long long T = 0;
+            for (int b = 0; b < a.B; ++b) T += (long long)plan_tiles[b] * a.Hkv * a.n_rb;
+            const int peff = plan_ctas(T, gridDim.x, a.min_tiles_per_cta);
+            const long long c = blockIdx.x;
+            s_peff = peff;
+            s_range[0] = c < peff ? cta_begin(c, T, peff) : 0;
+            s_range[1] = c < peff ? cta_begin(c + 1, T, peff) : 0;
+            for (int s = 0; s < NSTAGE; ++s) {
+                mbar_init(&full_bar[s], 1);
+                mbar_init(&empty_bar[s], NWC);
+            }
+            mbar_init(sync_bar, NWC);
+            fence_barrier_init();
+        }
+    }
+    __syncthreads();
+    const long long t_begin = s_range[0], t_end = s_range[1];
+    if (t_begin >= t_end) return;
+
+    if (warp == NWC) {
+        // =========================== producer warp =========================================
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+            const uint64_t pol = l2_evict_first_policy();
+            int b = 0;
+            long long b_start = 0;           // first flat tile of request b
+            long long per_b = (long long)plan_tiles[0] * a.Hkv * a.n_rb;
+            uint32_t it = 0;
+            for (long long t = t_begin; t < t_end; ++t, ++it) {
+                while (t >= b_start + per_b) {
+                    b_start += per_b;
+                    ++b;
+                    per_b = (long long)plan_tiles[b] * a.Hkv * a.n_rb;
+                }
+                const int nt_b = plan_tiles[b];
+                const long long off = t - b_start;
+                const int unit_in_b = (int)(off / nt_b);
+                const int tile = (int)(off - (long long)unit_in_b * nt_b);
+                const int h = unit_in_b / a.n_rb;
+                const int rb = unit_in_b - h * a.n_rb;
+                const long long u_start = b_start + (long long)unit_in_b * nt_b;
+                TileMeta m;
+                m.b = b; m.h = h; m.rb = rb;
+                m.unit = (b * a.Hkv + h) * a.n_rb + rb;
+                m.L_tot = plan_len[b];
+                m.flags = ((t == t_begin || tile == 0) ? kFirst : 0) |
+                          ((t == t_end - 1 || tile == nt_b - 1) ? kLast : 0) |
+                          ((u_start >= t_begin && u_start + nt_b <= t_end) ? kWhole : 0);
+                int ty = 0, tz = 0;
+                if (SRC == kSrcPaged) {
+                    const int page = tile < a.max_pages ? a.page_table[(size_t)b * a.max_pages + tile] : -1;
+                    m.pos0 = tile * kTileKeys;
+                    const int rem = m.L_tot - m.pos0;
+                    m.nvalid = rem < kTileKeys ? rem : kTileKeys;
+                    if (page < 0 || page >= a.num_pages) {
+                        flag_status(kStatusDeviceIndex);
+                        m.nvalid = 0;
+                    }
+                    ty = 0;
+                    tz = page * a.Hkv + h;
+                } else {
+                    Ranges r = ring_ranges(m.L_tot, a.n_sink, a.window, a.capacity);
+                    int tl = tile, k = 0;
+                    for (; k < r.n; ++k) {
+                        const int ntk = (r.len[k] + kTileKeys - 1) / kTileKeys;
+                        if (tl < ntk) break;
+                        tl -= ntk;
+                    }
+                    if (k >= r.n) k = r.n - 1;   // unreachable: tile < request_tiles
+                    const int rem = r.len[k] - tl * kTileKeys;
+                    m.pos0 = r.pos0[k] + tl * kTileKeys;
+                    m.nvalid = rem < kTileKeys ? rem : kTileKeys;
+                    ty = r.slot0[k] + tl * kTileKeys;
+                    tz = b * a.Hkv + h;
+                }
+                const int stage = (int)(it % NSTAGE);
+                const uint32_t phase = (it / NSTAGE) & 1u;
+                if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) break;
+                meta[stage] = m;
+                uint8_t* st = smem + (size_t)stage * kStageBytes;
+                if (m.nvalid > 0) {
+                    mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+                    tma_load_3d(st, &kmap, &full_bar[stage], 0, ty, tz, pol);
+                    tma_load_3d(st + kHalfBytes, &kmap, &full_bar[stage], 64, ty, tz, pol);
+                    tma_load_3d(st + kTileBytes, &vmap, &full_bar[stage], 0, ty, tz, pol);
+                    tma_load_3d(st + kTileBytes + kHalfBytes, &vmap, &full_bar[stage], 64, ty, tz, pol);
+                } else {
+                    mbar_arrive(&full_bar[stage]);
+                }
+            }
+            // Drain: wait (bounded) until the consumers released every stage, so no TMA copy is
+            // in flight into this CTA's shared memory when it exits.
+            const uint32_t issued = it;
+            for (uint32_t k = (issued > NSTAGE ? issued - NSTAGE : 0); k < issued; ++k) {
+                if (!mbar_wait_bounded(&empty_bar[k % NSTAGE], (k / NSTAGE) & 1u)) break;
+            }
+        }
+        return;
+    }
+
+    // ============================= consumer warps ==========================================
+    const int mt = warp % NMT;        // m-tile (16 rows)
+    const int kg = warp / NMT;        // key group
+    const int gid = lane >> 2, tig = lane & 3;
+    const int key0 = kg * KPW;
+
+    uint32_t qa[8][4];                // Q A-fragments, 8 k-steps of 16 dims
+    float o[16][4];                   // O accumulator: 16 n-tiles of 8 dims
+    float m_r[2], l_r[2];             // running max (log2 domain) and sum, rows gid / gid+8
+    unsigned long long vis[2];        // in-step visibility bitmask per row
+    int row_ok[2];
+    int Lpre = 0;
+
+    // per-lane ldmatrix row/chunk offsets
+    const int k_row_l = (lane & 7) + ((lane >> 4) << 3);   // K: matrices (n0,k0) (n0,k8) (n8,k0) (n8,k8)
+    const int k_chk_l = (lane >> 3) & 1;
+    const int v_row_l = (lane & 7) + (((lane >> 3) & 1) << 3);   // V^T: (k0,d0) (k8,d0) (k0,d8) (k8,d8)
+    const int v_chk_l = lane >> 4;
+
+    uint32_t it = 0;
+    uint32_t sync_phase = 0;
+    bool alive = true;
+    // Bounded rendezvous of the consumer warps (an mbarrier, so a sibling that gave up on a
+    // timed-out wait cannot leave the others blocked for ever).
+    auto consumers_sync = [&]() -> bool {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sync_bar);
+        const bool ok = mbar_wait_bounded(sync_bar, sync_phase);
+        sync_phase ^= 1u;
+        return ok;
+    };
+    for (long long t = t_begin; t < t_end && alive; ++t, ++it) {
+        const int stage = (int)(it % NSTAGE);
+        const uint32_t phase = (it / NSTAGE) & 1u;
+        if (!mbar_wait_bounded(&full_bar[stage], phase)) { alive = false; break; }
+        const TileMeta m = meta[stage];
+
+        if (m.flags & kFirst) {
+            // ---- unit start: load this warp's Q rows, visibility masks, reset state -------
+            Lpre = m.L_tot - a.n_q;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
+                row_ok[r] = R < a.rows_total;
+                const int i = row_ok[r] ? R / a.G : 0;
+                unsigned long long msk = 0ull;
+                if (a.tree_parent != nullptr) {
+                    int cur = i;
+                    for (int k = 0; k < 64 && cur >= 0 && cur < a.n_q; ++k) {
+                        msk |= 1ull << cur;
+                        const int nxt = a.tree_parent[(size_t)m.b * a.n_q + cur];
+                        cur = (nxt < cur) ? nxt : -1;
+                    }
+                } else {
+                    msk = (i >= 63) ? ~0ull : ((1ull << (i + 1)) - 1ull);
+                }
+                vis[r] = msk;
+                m_r[r] = -INFINITY;
+                l_r[r] = 0.f;
+            }
+#pragma unroll
+            for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            const uint32_t* q32[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
+                const int i = R / a.G, g = R - (R / a.G) * a.G;
+                q32[r] = reinterpret_cast<const uint32_t*>(
+                    a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int c = ks * 8 + tig;     // 32-bit word index of dims (16 ks + 2 tig)
+                qa[ks][0] = row_ok[0] ? __ldg(q32[0] + c) : 0u;
+                qa[ks][1] = row_ok[1] ? __ldg(q32[1] + c) : 0u;
+                qa[ks][2] = row_ok[0] ? __ldg(q32[0] + c + 4) : 0u;
+                qa[ks][3] = row_ok[1] ? __ldg(q32[1] + c + 4) : 0u;
+            }
+        }
+
+        if (m.nvalid > 0) {
+            const uint32_t kbase = smem_addr(smem + (size_t)stage * kStageBytes);
+            const uint32_t vbase = kbase + kTileBytes;
+            // ---- S = Q K^T over this warp's KPW keys -------------------------------------
+            float s[NT][4];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                for (int np = 0; np < NT / 2; ++np) {
+                    uint32_t b0a, b1a, b0b, b1b;
+                    ldsm_x4(tile_chunk_addr(kbase, key0 + np * 16 + k_row_l, ks * 2 + k_chk_l),
+                            b0a, b1a, b0b, b1b);
+                    mma_bf16_16816(s[2 * np], qa[ks], b0a, b1a);
+                    mma_bf16_16816(s[2 * np + 1], qa[ks], b0b, b1b);
+                }
+            }
+            // ---- mask: ragged tile end, in-step (causal / tree) keys ----------------------
+            const bool need_mask = (m.nvalid < kTileKeys) || (m.pos0 + kTileKeys > Lpre);
+            if (need_mask) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int kr = key0 + n * 8 + 2 * tig + (e & 1);
+                        const int pos = m.pos0 + kr;
+                        const int off = pos - Lpre;
+                        const unsigned long long vm = vis[e >> 1];
+                        const bool ok = kr < m.nvalid &&
+                                        (off < 0 || (off < 64 && ((vm >> off) & 1ull)));
+                        if (!ok) s[n][e] = -INFINITY;
+                    }
+                }
+            }
+            // ---- online softmax (base 2) -------------------------------------------------
+            uint32_t pa[NT / 2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m_r[r], mx * a.scale_log2);
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = fast_exp2(m_r[r] - m_use);
+                m_r[r] = m_new;
+                l_r[r] *= alpha;
+#pragma unroll
+                for (int n = 0; n < 16; ++n) { o[n][2 * r] *= alpha; o[n][2 * r + 1] *= alpha; }
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const float p0 = fast_exp2(fmaf(s[n][2 * r], a.scale_log2, -m_use));
+                    const float p1 = fast_exp2(fmaf(s[n][2 * r + 1], a.scale_log2, -m_use));
+                    const uint32_t pk = pack_bf16x2(p0, p1);
+                    // the row sum uses the same bf16-rounded weights the PV product uses
+                    l_r[r] += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+                    pa[n >> 1][r + 2 * (n & 1)] = pk;
+                }
+            }
+            // ---- O += P V ------------------------------------------------------------------
+            const bool ragged = m.nvalid < kTileKeys;
+#pragma unroll
+            for (int kk = 0; kk < NT / 2; ++kk) {
+                const int krow = key0 + kk * 16;
+                uint32_t lo_keep = 0xffffffffu, hi_keep = 0xffffffffu;   // keys 2tig(+1), +8
+                if (ragged) {
+                    const int k0 = krow + 2 * tig;
+                    lo_keep = (k0 < m.nvalid ? 0x0000ffffu : 0u) | (k0 + 1 < m.nvalid ? 0xffff0000u : 0u);
+                    hi_keep = (k0 + 8 < m.nvalid ? 0x0000ffffu : 0u) | (k0 + 9 < m.nvalid ? 0xffff0000u : 0u);
+                }
+#pragma unroll
+                for (int dp = 0; dp < 8; ++dp) {
+                    uint32_t b0a, b1a, b0b, b1b;
+                    ldsm_x4_trans(tile_chunk_addr(vbase, krow + v_row_l, dp * 2 + v_chk_l),
+                                  b0a, b1a, b0b, b1b);
+                    if (ragged) {
+                        b0a &= lo_keep; b0b &= lo_keep;
+                        b1a &= hi_keep; b1b &= hi_keep;
+                    }
+                    mma_bf16_16816(o[2 * dp], pa[kk], b0a, b1a);
+                    mma_bf16_16816(o[2 * dp + 1], pa[kk], b0b, b1b);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[stage]);
+
+        if (m.flags & kLast) {
+            // ---- unit end: combine key groups, then write the result or a partial ----------
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 1);
+                l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 2);
+            }
+            if (NKG > 1) {
+                if (kg > 0) {
+                    float* mo = merge_o + ((size_t)((kg - 1) * NMT + mt) * 16) * L::kMergeStride;
+                    float* ml = merge_ml + ((size_t)((kg - 1) * NMT + mt) * 16) * 2;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int row = gid + 8 * r;
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            *reinterpret_cast<float2*>(mo + row * L::kMergeStride + n * 8 + 2 * tig) =
+                                make_float2(o[n][2 * r], o[n][2 * r + 1]);
+                        if (tig == 0) { ml[row * 2] = m_r[r]; ml[row * 2 + 1] = l_r[r]; }
+                    }
+                }
+                if (!consumers_sync()) { alive = false; break; }
+                if (kg == 0) {
+#pragma unroll 1
+                    for (int g2 = 1; g2 < NKG; ++g2) {
+                        const float* mo = merge_o + ((size_t)((g2 - 1) * NMT + mt) * 16) * L::kMergeStride;
+                        const float* ml = merge_ml + ((size_t)((g2 - 1) * NMT + mt) * 16) * 2;
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int row = gid + 8 * r;
+                            const float m2 = ml[row * 2], l2 = ml[row * 2 + 1];
+                            const float mn = fmaxf(m_r[r], m2);
+                            const float mu = (mn == -INFINITY) ? 0.f : mn;
+                            const float w1 = fast_exp2(m_r[r] - mu), w2 = fast_exp2(m2 - mu);
+                            l_r[r] = l_r[r] * w1 + l2 * w2;
+                            m_r[r] = mn;
+#pragma unroll
+                            for (int n = 0; n < 16; ++n) {
+                                const float2 v2 = *reinterpret_cast<const float2*>(
+                                    mo + row * L::kMergeStride + n * 8 + 2 * tig);
+                                o[n][2 * r] = o[n][2 * r] * w1 + v2.x * w2;
+                                o[n][2 * r + 1] = o[n][2 * r + 1] * w1 + v2.y * w2;
+                            }
+                        }
+                    }
+                }
+                if (!consumers_sync()) { alive = false; break; }
+            }
+            if (kg == 0) {
+                const int slot = (int)blockIdx.x + m.unit;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    if (!row_ok[r]) continue;
+                    const int rr = mt * 16 + gid + 8 * r;            // row within the block
+                    const int R = m.rb * kRowsPerBlock + rr;
+                    const float l = l_r[r];
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    const float lse2 = l > 0.f ? m_r[r] + __log2f(l) : -INFINITY;
+                    if (m.flags & kWhole) {
+                        const int i = R / a.G, g = R - (R / a.G) * a.G;
+                        const size_t orow = ((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g;
+                        uint32_t* op = reinterpret_cast<uint32_t*>(a.out + orow * kD);
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            op[n * 4 + tig] = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+                        if (a.lse != nullptr && tig == 0) a.lse[orow] = lse2 * kLn2;
+                    } else {
+                        float* wo = a.ws_o + ((size_t)slot * kRowsPerBlock + rr) * kD;
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            *reinterpret_cast<float2*>(wo + n * 8 + 2 * tig) =
+                                make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+                        if (tig == 0) a.ws_lse[(size_t)slot * kRowsPerBlock + rr] = lse2;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// lse_merge_kernel: combines the split partials of units that span several CTAs, and writes
+// empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block), 128
+// threads (one per head dim).  Partial s has weight 2^(lse_s - max_s lse_s); empty partials have
+// lse = -inf and weight 0.
+template <int SRC>
+__global__ void __launch_bounds__(kD)
+lse_merge_kernel(const AttnArgs a, int P_launch) {
+    const int u = blockIdx.x;
+    const int rr = blockIdx.y;
+    const int rb = u % a.n_rb;
+    const int h = (u / a.n_rb) % a.Hkv;
+    const int b = u / (a.n_rb * a.Hkv);
+    const int R = rb * kRowsPerBlock + rr;
+    if (R >= a.rows_total) return;
+
+    __shared__ long long s_info[3];     // T, unit start, unit tiles
+    if (threadIdx.x == 0) {
+        long long T = 0, start = 0;
+        int nt_u = 0;
+        for (int bb = 0; bb < a.B; ++bb) {
+            const int nt = request_tiles<SRC>(a, request_len<SRC>(a, bb));
+            if (bb == b) { start = T + (long long)(h * a.n_rb + rb) * nt; nt_u = nt; }
+            T += (long long)nt * a.Hkv * a.n_rb;
+        }
+        s_info[0] = T; s_info[1] = start; s_info[2] = nt_u;
+    }
+    __syncthreads();
+    const long long T = s_info[0], start = s_info[1];
+    const int nt_u = (int)s_info[2];
+    const int i = R / a.G, g = R - (R / a.G) * a.G;
+    const size_t orow = ((size_t)b * a.n_q + i) * a.Hq + (size_t)h * a.G + g;
+    const int d = threadIdx.x;
+    if (nt_u == 0) {
+        a.out[orow * kD + d] = __float2bfloat16_rn(0.f);
+        if (a.lse != nullptr && d == 0) a.lse[orow] = -INFINITY;
+        return;
+    }
+    const int peff = plan_ctas(T, P_launch, a.min_tiles_per_cta);
+    const int c_lo = cta_of_tile(start, T, peff);
+    const int c_hi = cta_of_tile(start + nt_u - 1, T, peff);
+    if (c_lo == c_hi) return;           // finished inside one CTA
+    float mx = -INFINITY;
+    for (int c = c_lo; c <= c_hi; ++c)
+        mx = fmaxf(mx, a.ws_lse[(size_t)(c + u) * kRowsPerBlock + rr]);
+    float acc = 0.f, wsum = 0.f;
+    if (mx != -INFINITY) {
+        for (int c = c_lo; c <= c_hi; ++c) {
+            const size_t slot = (size_t)(c + u);
+            const float w = exp2f(a.ws_lse[slot * kRowsPerBlock + rr] - mx);
+            wsum += w;
+            acc += w * a.ws_o[(slot * kRowsPerBlock + rr) * kD + d];
+        }
+    }
+    const float res = wsum > 0.f ? acc / wsum : 0.f;
+    a.out[orow * kD + d] = __float2bfloat16_rn(res);
+    if (a.lse != nullptr && d == 0) a.lse[orow] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
+}
+
+}  // namespace wmtp

@@ -1,0 +1,347 @@
+// capi.cu -- the C ABI of libwmtp.so (declared in include/wmtp.h): host-side argument checks,
+// TMA tensor-map encoding, workspace layout and kernel launches.  One translation unit holds all
+// device code, so the device status word needs no relocatable device code.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "wmtp.h"
+#include "attn_kernels.cuh"
+#include "ring_accept_kernels.cuh"
+
+namespace wmtp {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0;
+    bool ok = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_done[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device(int* dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) return WMTP_ERR_CUDA;
+    if (*dev < 0 || *dev >= kMaxDevices) return WMTP_ERR_CUDA;
+    return WMTP_OK;
+}
+
+int device_info(DeviceInfo* out) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc != WMTP_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev_done[dev]) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return WMTP_ERR_CUDA;
+        d.ok = (d.major == 10);
+        g_dev[dev] = d;
+        g_dev_done[dev] = true;
+    }
+    *out = g_dev[dev];
+    return out->ok ? WMTP_OK : WMTP_ERR_UNSUPPORTED;
+}
+
+int encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || p == nullptr)
+            return WMTP_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    *fn = g_encode;
+    return WMTP_OK;
+}
+
+// A [n_blocks][rows][128] bf16 tensor viewed as 3-D (dim, row, block), read in 64x64 boxes with
+// the 128-byte swizzle.  Rows past `rows` and blocks past `n_blocks` read as zero.
+int encode_rows_map(CUtensorMap* map, const void* base, long long rows, long long n_blocks) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int rc = encoder(&enc);
+    if (rc != WMTP_OK) return rc;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)n_blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int min_tiles_per_cta() {
+    static int v = [] {
+        const char* e = std::getenv("WMTP_MIN_TILES");
+        int x = e ? std::atoi(e) : 2;
+        return x < 1 ? 1 : x;
+    }();
+    return v;
+}
+
+struct Shape {
+    int B, n_q, Hq, Hkv, G, rows_total, rows_blk, n_rb, units;
+};
+
+int check_shape(int B, int n_q, int Hq, int Hkv, int D, Shape* s) {
+    if (B < 1 || n_q < 1 || Hq < 1 || Hkv < 1) return WMTP_ERR_ARG;
+    if (D != WMTP_HEAD_DIM) return WMTP_ERR_SHAPE;
+    if (Hq % Hkv != 0 || Hq / Hkv > WMTP_MAX_GROUP || n_q > WMTP_MAX_QUERIES || B > kMaxBatch)
+        return WMTP_ERR_SHAPE;
+    s->B = B; s->n_q = n_q; s->Hq = Hq; s->Hkv = Hkv; s->G = Hq / Hkv;
+    s->rows_total = n_q * s->G;
+    s->rows_blk = s->rows_total < kRowsPerBlock ? s->rows_total : kRowsPerBlock;
+    s->n_rb = (s->rows_total + kRowsPerBlock - 1) / kRowsPerBlock;
+    s->units = B * Hkv * s->n_rb;
+    return WMTP_OK;
+}
+
+// Workspace: [slots][64][128] fp32 partial outputs, then [slots][64] fp32 partial LSEs.
+size_t ws_o_bytes(long long slots) { return (size_t)slots * kRowsPerBlock * kD * sizeof(float); }
+size_t ws_total_bytes(long long slots) {
+    size_t a = (ws_o_bytes(slots) + 255) & ~size_t(255);
+    return a + (size_t)slots * kRowsPerBlock * sizeof(float);
+}
+
+constexpr int kStages = 4;
+
+template <int SRC, int NMT, int NKG>
+int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int grid,
+                  const Shape& s, cudaStream_t st) {
+    using Lay = SmemLayout<NMT, NKG, kStages>;
+    auto kern = attn_split_kernel<SRC, NMT, NKG, kStages>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev;
+    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess)
+            return WMTP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    kern<<<grid, (NMT * NKG + 1) * 32, Lay::kAlloc, st>>>(km, vm, a);
+    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    lse_merge_kernel<SRC><<<dim3(s.units, s.rows_blk), kD, 0, st>>>(a, grid);
+    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    return WMTP_OK;
+}
+
+template <int SRC>
+int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int grid,
+                const Shape& s, cudaStream_t st) {
+    const int nmt = (s.rows_blk + 15) / 16;
+    switch (nmt) {
+        case 1: return launch_attn_t<SRC, 1, 4>(km, vm, a, grid, s, st);
+        case 2: return launch_attn_t<SRC, 2, 2>(km, vm, a, grid, s, st);
+        case 3: return launch_attn_t<SRC, 3, 2>(km, vm, a, grid, s, st);
+        default: return launch_attn_t<SRC, 4, 2>(km, vm, a, grid, s, st);
+    }
+}
+
+// Common front half of the three attention calls.
+int prepare(const Shape& s, const void* q, const void* out, const float* lse, void* ws,
+            size_t ws_bytes, float sm_scale, DeviceInfo* dev, AttnArgs* a) {
+    if (q == nullptr || out == nullptr || ws == nullptr) return WMTP_ERR_ARG;
+    if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return WMTP_ERR_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || (lse && !aligned(lse, 4)) || !aligned(ws, 256))
+        return WMTP_ERR_ALIGN;
+    int rc = device_info(dev);
+    if (rc != WMTP_OK) return rc;
+    const long long slots = (long long)dev->sm_count + s.units;
+    if (ws_bytes < ws_total_bytes(slots)) return WMTP_ERR_WORKSPACE;
+    std::memset(a, 0, sizeof(*a));
+    a->q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a->out = reinterpret_cast<__nv_bfloat16*>(const_cast<void*>(out));
+    a->lse = const_cast<float*>(lse);
+    a->ws_o = reinterpret_cast<float*>(ws);
+    a->ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
+                                         ((ws_o_bytes(slots) + 255) & ~size_t(255)));
+    a->B = s.B; a->n_q = s.n_q; a->Hq = s.Hq; a->Hkv = s.Hkv; a->G = s.G; a->n_rb = s.n_rb;
+    a->rows_total = s.rows_total;
+    a->scale_log2 = sm_scale * 1.4426950408889634f;
+    a->min_tiles_per_cta = min_tiles_per_cta();
+    return WMTP_OK;
+}
+
+int paged_call(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_pool,
+               const int32_t* page_table, const int32_t* kv_len, const int32_t* tree_parent,
+               int B, int n_q, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages,
+               float sm_scale, wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+               cudaStream_t st) {
+    Shape s;
+    int rc = check_shape(B, n_q, Hq, Hkv, D, &s);
+    if (rc != WMTP_OK) return rc;
+    if (page_size != WMTP_PAGE_SIZE) return WMTP_ERR_SHAPE;
+    if (k_pool == nullptr || v_pool == nullptr || page_table == nullptr || kv_len == nullptr)
+        return WMTP_ERR_ARG;
+    if (max_pages < 1 || num_pages < 1) return WMTP_ERR_ARG;
+    if ((long long)num_pages * Hkv > 0x7fffffffll) return WMTP_ERR_SHAPE;
+    if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(page_table, 4) ||
+        !aligned(kv_len, 4) || (tree_parent && !aligned(tree_parent, 4)))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    AttnArgs a;
+    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a);
+    if (rc != WMTP_OK) return rc;
+    a.tree_parent = tree_parent;
+    a.page_table = page_table;
+    a.kv_len = kv_len;
+    a.max_pages = max_pages;
+    a.num_pages = num_pages;
+    CUtensorMap km, vm;
+    if ((rc = encode_rows_map(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
+    if ((rc = encode_rows_map(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
+    return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st);
+}
+
+}  // namespace
+}  // namespace wmtp
+
+using namespace wmtp;
+
+extern "C" {
+
+const char* wmtp_status_string(int status) {
+    switch (status) {
+        case WMTP_OK: return "ok";
+        case WMTP_ERR_ARG: return "invalid argument";
+        case WMTP_ERR_SHAPE: return "unsupported shape";
+        case WMTP_ERR_ALIGN: return "misaligned pointer";
+        case WMTP_ERR_WORKSPACE: return "workspace too small";
+        case WMTP_ERR_CUDA: return "CUDA error";
+        case WMTP_ERR_DEVICE_INDEX: return "device-side index out of range";
+        case WMTP_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
+        case WMTP_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+size_t wmtp_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D) {
+    Shape s;
+    if (check_shape(B, n_q, Hq, Hkv, D, &s) != WMTP_OK) return 0;
+    DeviceInfo dev;
+    if (device_info(&dev) != WMTP_OK) return 0;
+    return ws_total_bytes((long long)dev.sm_count + s.units);
+}
+
+int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, const wmtp_bf16* k_new,
+                   const wmtp_bf16* v_new, int B, int n_new, int Hkv, int D, int n_sink, int capacity,
+                   wmtp_stream_t stream) {
+    if (ring_k == nullptr || ring_v == nullptr || ring_len == nullptr) return WMTP_ERR_ARG;
+    if (B < 1 || n_new < 0 || Hkv < 1 || n_sink < 0 || capacity <= n_sink) return WMTP_ERR_ARG;
+    if (D != WMTP_HEAD_DIM) return WMTP_ERR_SHAPE;
+    if (B > 65535) return WMTP_ERR_SHAPE;                      // grid.y
+    if (n_new == 0) return WMTP_OK;
+    if (k_new == nullptr || v_new == nullptr) return WMTP_ERR_ARG;
+    if (!aligned(ring_k, 16) || !aligned(ring_v, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+        !aligned(ring_len, 8))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // upper bound on surviving rows per request: the sink plus the ring's other slots
+    const long long surv = (long long)(n_new < capacity ? n_new : capacity);
+    const long long work = surv * Hkv * 16;
+    long long chunks = (work + 256 * 4 - 1) / (256 * 4);     // ~4 pieces per thread
+    const long long max_chunks = (long long)dev.sm_count * 8;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    const int single = (chunks == 1);
+    ring_append_kernel<<<dim3((unsigned)chunks, B), 256, 0, st>>>(
+        reinterpret_cast<uint4*>(ring_k), reinterpret_cast<uint4*>(ring_v),
+        reinterpret_cast<long long*>(ring_len), reinterpret_cast<const uint4*>(k_new),
+        reinterpret_cast<const uint4*>(v_new), n_new, Hkv, n_sink, capacity, single);
+    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    if (!single) {
+        ring_len_add_kernel<<<(B + 255) / 256, 256, 0, st>>>(reinterpret_cast<long long*>(ring_len), B, n_new);
+        if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    }
+    return WMTP_OK;
+}
+
+int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,
+                      const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D, int n_sink,
+                      int window, int capacity, float sm_scale, wmtp_bf16* out, float* lse, void* ws,
+                      size_t ws_bytes, wmtp_stream_t stream) {
+    Shape s;
+    int rc = check_shape(B, n_q, Hq, Hkv, D, &s);
+    if (rc != WMTP_OK) return rc;
+    if (ring_k == nullptr || ring_v == nullptr || ring_len == nullptr) return WMTP_ERR_ARG;
+    if (n_sink < 0 || window < 0 || capacity <= n_sink || window > capacity - n_sink) return WMTP_ERR_ARG;
+    if ((long long)B * Hkv > 0x7fffffffll) return WMTP_ERR_SHAPE;
+    if (!aligned(ring_k, 16) || !aligned(ring_v, 16) || !aligned(ring_len, 8)) return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    AttnArgs a;
+    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a);
+    if (rc != WMTP_OK) return rc;
+    a.ring_len = reinterpret_cast<const long long*>(ring_len);
+    a.n_sink = n_sink;
+    a.window = window;
+    a.capacity = capacity;
+    CUtensorMap km, vm;
+    if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
+    if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
+    return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int draft_attn_full(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_pool,
+                    const int32_t* page_table, const int32_t* kv_len, int B, int n_q, int Hq, int Hkv,
+                    int D, int page_size, int max_pages, int num_pages, float sm_scale, wmtp_bf16* out,
+                    float* lse, void* ws, size_t ws_bytes, wmtp_stream_t stream) {
+    return paged_call(q, k_pool, v_pool, page_table, kv_len, nullptr, B, n_q, Hq, Hkv, D, page_size,
+                      max_pages, num_pages, sm_scale, out, lse, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int verify_attn(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_pool,
+                const int32_t* page_table, const int32_t* kv_len, const int32_t* tree_parent, int B,
+                int n_q, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages,
+                float sm_scale, wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                wmtp_stream_t stream) {
+    return paged_call(q, k_pool, v_pool, page_table, kv_len, tree_parent, B, n_q, Hq, Hkv, D,
+                      page_size, max_pages, num_pages, sm_scale, out, lse, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int accept_greedy(const float* logits, const int32_t* tokens, const int32_t* tree_parent, int B,
+                  int n_q, int V, int32_t* accepted, int32_t* n_accepted, wmtp_stream_t stream) {
+    if (logits == nullptr || tokens == nullptr || accepted == nullptr || n_accepted == nullptr)
+        return WMTP_ERR_ARG;
+    if (B < 1 || n_q < 1 || V < 1 || n_q > WMTP_MAX_QUERIES) return WMTP_ERR_ARG;
+    if (!aligned(logits, 4) || !aligned(tokens, 4) || !aligned(accepted, 4) || !aligned(n_accepted, 4) ||
+        (tree_parent && !aligned(tree_parent, 4)))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    accept_greedy_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        logits, tokens, tree_parent, n_q, V, accepted, n_accepted);
+    return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+}
+
+int wmtp_device_status(wmtp_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return WMTP_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return WMTP_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return WMTP_ERR_CUDA;
+    if (v & kStatusDeviceIndex) return WMTP_ERR_DEVICE_INDEX;
+    if (v & kStatusTimeout) return WMTP_ERR_TIMEOUT;
+    return WMTP_OK;
+}
+
+}  // extern "C"
