@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of the Windowed-MTP decode step on B200: microseconds per decode step and KV-read
+GB/s against the measured HBM peak, windowed vs native full-context draft, at 1M context.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ctx1m] [--gamma 3]
+    python bench.py --impl reference ...      # the fp64 CPU oracle as the reference arm
+
+One step = the whole hot path once (Pith verdict on arXiv 2607.21535, Eq. 1): the draft's
+context pass and gamma draft forwards (ring append + windowed attention, or full paged attention
+in the native arm), verify attention over every target attention layer, greedy acceptance.
+Inputs are synthetic and resident in HBM before timing; each step streams ~26 GiB of KV
+(more than the 126 MB L2), so no L2 flush is needed between steps.  Rank 0 prints one JSON line.
+With N GPUs every rank runs an independent replica (the path has no exchange step).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs per decode step & KV-read GB/s vs HBM peak at 1M ctx (windowed vs full draft)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="wmtp", choices=["wmtp", "reference"])
+    p.add_argument("--workload", default="ctx1m")
+    p.add_argument("--gamma", type=int, default=3)
+    p.add_argument("--window", type=int, default=0, help="recent window W (default: the workload's first)")
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- environment
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_speculative_kv_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[0] == kernel \
+                    and parts[1] == workload and parts[3] == src:
+                return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of one GPU while the timed region runs (started before, stopped after)."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.count(",") >= 6]
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_speculative_kv_b200 import accounting as acc
+    from long_context_speculative_kv_b200 import api
+    from long_context_speculative_kv_b200.step import CallLog, DecodeStep, StepBuffers
+    from synthetic import configs, workload
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = configs.BY_NAME[args.workload]
+    window = args.window or w.windows[0]
+    gammas = sorted(set(w.gammas) | {args.gamma}) if not args.no_sweep else [args.gamma]
+    if w.tree_nodes:
+        gammas = [args.gamma]
+    max_nq = max([w.tree_nodes or (g + 1) for g in gammas])
+    shared = workload.shared_inputs(w, device, max_nq_verify=max_nq, max_gamma=max(gammas),
+                                    window=window)
+    lens = shared["lens"]
+    Lsum = sum(lens)
+
+    def make_step(gamma):
+        return DecodeStep(StepBuffers(**workload.step_inputs(w, shared, gamma, device)), gamma)
+
+    step = make_step(args.gamma)
+    n_q_v = step.n_q_verify
+    n_layers = step.n_layers
+
+    # ---- algorithmic bytes per call (KV only) -------------------------------------------
+    row = acc.kv_row_bytes(w.Hkv, w.D)
+    bytes_verify = sum(L + n_q_v for L in lens) * row
+    bytes_full_fwd = sum(L + args.gamma + 2 for L in lens) * row        # last forward's length
+    bytes_full_ctx = sum(L + args.gamma + 1 for L in lens) * row
+    bytes_window = sum(acc.window_keys(L + args.gamma + 1, w.n_sink, window) for L in lens) * row
+
+    for _ in range(args.warmup):
+        step.run("windowed")
+        step.run("native")
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+
+    def timed(arm, K, with_log=True, e2e=None):
+        logs = []
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0 = api.launch_count()
+        e0.record()
+        for _ in range(K):
+            if e2e is not None:
+                step.run_e2e(arm, *e2e)
+            else:
+                log = CallLog() if with_log else None
+                step.run(arm, log)
+                logs.append(log)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        return e0.elapsed_time(e1), logs, api.launch_count() - n0
+
+    props = torch.cuda.get_device_properties(device)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    clocks = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    ms_w, logs_w, launches = timed("windowed", args.steps)
+    ms_n, logs_n, _ = timed("native", args.steps)
+    clk = clocks.stop()
+    assert api.device_status() == 0
+
+    def per_label(logs):
+        d = {}
+        for lg in logs:
+            for lab, ms in lg.durations_ms():
+                d.setdefault(lab, []).append(ms)
+        return d
+
+    def phases(logs, draft_labels):
+        t_d, t_v, t_a = [], [], []
+        for lg in logs:
+            dur = lg.durations_ms()
+            t_d.append(sum(ms for lab, ms in dur if lab in draft_labels))
+            t_v.append(sum(ms for lab, ms in dur if lab == "verify"))
+            t_a.append(sum(ms for lab, ms in dur if lab == "accept"))
+        return statistics.mean(t_d) * 1e3, statistics.mean(t_v) * 1e3, statistics.mean(t_a) * 1e3
+
+    lw, ln = per_label(logs_w), per_label(logs_n)
+    us_w_local = ms_w * 1e3 / args.steps
+    us_n_local = ms_n * 1e3 / args.steps
+    ms_w_max, ms_n_max = max_ranks(ms_w), max_ranks(ms_n)
+    value = ms_w_max * 1e3 / (args.steps * world)          # aggregate: all ranks' steps
+    tdw, tvw, taw = phases(logs_w, {"append_ctx", "window_ctx", "append_fwd", "window_fwd"})
+    tdn, tvn, tan = phases(logs_n, {"full_ctx", "full_fwd"})
+
+    peaks = measured_peaks()
+    hbm = peaks["hbm_gbs"]
+
+    def kstat(label_times, nbytes):
+        if not label_times:
+            return None
+        us = statistics.mean(label_times) * 1e3
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": round(us, 3), "us_median": round(statistics.median(label_times) * 1e3, 3),
+                "bytes": nbytes, "GBps": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm, 4)}
+
+    kernels = {
+        "verify_attn": kstat(lw.get("verify"), bytes_verify),
+        "draft_attn_full_fwd": kstat(ln.get("full_fwd"), bytes_full_fwd),
+        "draft_attn_full_ctx": kstat(ln.get("full_ctx"), bytes_full_ctx),
+        "draft_attn_window_fwd_inloop": kstat(lw.get("window_fwd"), bytes_window),
+        "draft_attn_window_ctx_inloop": kstat(lw.get("window_ctx"), bytes_window),
+        "ring_kv_append_1": kstat(lw.get("append_fwd"), acc.append_bytes(1, w.Hkv, w.D) * w.B),
+        "accept_greedy": kstat(lw.get("accept"), w.B * n_q_v * w.vocab * 4),
+    }
+
+    # ---- windowed draft with a cold L2: rotate over ring copies larger than 2x L2 ----------
+    cold = None
+    if "ring_k" in shared:
+        l2 = props.L2_cache_size if hasattr(props, "L2_cache_size") else 126 << 20
+        ring_bytes = shared["ring_k"].numel() * 4
+        R = max(4, int(2.5 * l2 // ring_bytes) + 1)
+        rings = [(torch.empty_like(shared["ring_k"]).normal_(), torch.empty_like(shared["ring_v"]).normal_())
+                 for _ in range(R)]
+        rl = shared["ring_len0"] + args.gamma + 2
+        b = step.b
+        times = []
+        for it in range(3 * R):
+            rk, rv = rings[it % R]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            api.draft_attn_window(b.q_fwd[0], rk, rv, rl, w.n_sink, window, w.sm_scale, b.ws,
+                                  out=b.out["fwd"], lse=b.out["fwd_lse"])
+            e1.record()
+            times.append((e0, e1))
+        torch.cuda.synchronize()
+        t = [a.elapsed_time(c) for a, c in times[R:]]
+        cold = kstat(t, bytes_window)
+        cold["rotating_copies"] = R
+        del rings
+        torch.cuda.empty_cache()
+
+    # ---- end to end through the public API with host buffers --------------------------------
+    h_in, h_out = step.host_inputs(), step.host_outputs()
+    for _ in range(2):
+        step.run_e2e("windowed", h_in, h_out)
+    ms_e2e, _, _ = timed("windowed", args.steps, e2e=(h_in, h_out))
+    e2e_value = max_ranks(ms_e2e) * 1e3 / (args.steps * world)
+
+    # ---- draft-depth sweep -------------------------------------------------------------
+    sweep = {}
+    if len(gammas) > 1:
+        Ks = max(5, args.steps // 10)
+        base_step = step
+        for g in gammas:
+            step = base_step if g == args.gamma else make_step(g)
+            for _ in range(2):
+                step.run("windowed")
+                step.run("native")
+            mw, lgw, _ = timed("windowed", Ks)
+            mn, lgn, _ = timed("native", Ks)
+            dw, vw, _ = phases(lgw, {"append_ctx", "window_ctx", "append_fwd", "window_fwd"})
+            dn, vn, _ = phases(lgn, {"full_ctx", "full_fwd"})
+            sweep[str(g)] = {"windowed_us": round(max_ranks(mw) * 1e3 / Ks, 2),
+                             "native_us": round(max_ranks(mn) * 1e3 / Ks, 2),
+                             "t_draft_windowed_us": round(dw, 2), "t_draft_native_us": round(dn, 2),
+                             "t_verify_us": round((vw + vn) / 2, 2)}
+            sweep[str(g)]["step_cost_reduction_pct"] = round(
+                100 * (sweep[str(g)]["native_us"] / sweep[str(g)]["windowed_us"] - 1), 2)
+        step = base_step
+
+    # ---- KV accounting -------------------------------------------------------------------
+    sb_w = acc.step_bytes(int(statistics.mean(lens)), args.gamma, n_q_v, w.Hkv, w.D, n_layers,
+                          w.n_sink, window, windowed=True)
+    sb_n = acc.step_bytes(int(statistics.mean(lens)), args.gamma, n_q_v, w.Hkv, w.D, n_layers,
+                          w.n_sink, window, windowed=False)
+    Lm = int(statistics.mean(lens))
+    accounting = {
+        "draft_kv_bytes_per_step_windowed": sb_w.draft * w.B,
+        "draft_kv_bytes_per_step_native": sb_n.draft * w.B,
+        "draft_kv_entries_dropped": round(acc.dropped_fraction(Lm, w.n_sink + window), 6),
+        "kv_reclaimed_share_of_total": round(acc.reclaimed_share_of_total(Lm, w.n_sink + window, n_layers), 6),
+        "pages_quote": "+28% to +44% per-decode-step cost reduction at 1M, ~99% draft KV dropped, "
+                       "7.7-11% of total KV reclaimed (one GPU in SGLang, hardware unstated)",
+    }
+
+    # ---- CPU baseline: the oracle on the host cores (rank 0, one GPU only) ------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_step_estimate(w, args.gamma, window, lens, n_q_v, n_layers)
+
+    traffic = committed_traffic("verify_attn", w.name)
+    v = kernels["verify_attn"]
+    roofline = {"kernel": "verify_attn (split attention + LSE merge, one target layer)",
+                "bound": "hbm", "achieved": v["GBps"], "peak": hbm, "unit": "GB/s",
+                "frac": v["frac_of_hbm_peak"],
+                "traffic": traffic, "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
+
+    cfg = {"workload": f"{w.name}: B={w.B} L={'ragged ' + str(w.ragged) if w.ragged[1] else w.L} "
+                       f"Hq={w.Hq} Hkv={w.Hkv} D={w.D} page={w.page_size} window={w.n_sink}+{window} "
+                       f"gamma={args.gamma} verify_layers={n_layers}"
+                       + (f" tree={w.tree_nodes}" if w.tree_nodes else " chain"),
+           "gamma": args.gamma, "window": window, "n_sink": w.n_sink, "verify_layers": n_layers,
+           "batch": w.B, "context": lens if w.B <= 8 else Lm,
+           "l2": "inputs larger than L2 (each step streams %.1f GiB of KV)" % (sb_w.total * w.B / 2 ** 30),
+           "value_is": "windowed-arm us per decode step = max-over-ranks time / (steps x ranks)",
+           "parallelism": f"replicas x{world}"}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "us/step", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1e3, 6),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V, random page tables)", "config": cfg,
+        "windowed": {"us_per_step": round(us_w_local, 2), "t_draft_us": round(tdw, 2),
+                     "t_verify_us": round(tvw, 2), "t_accept_us": round(taw, 2)},
+        "native": {"us_per_step": round(us_n_local, 2), "t_draft_us": round(tdn, 2),
+                   "t_verify_us": round(tvn, 2), "t_accept_us": round(tan, 2)},
+        "step_cost_ratio_native_over_windowed": round(ms_n_max / ms_w_max, 4),
+        "step_cost_reduction_pct": round(100 * (ms_n_max / ms_w_max - 1), 2),
+        "kernels": dict(kernels, draft_attn_window_fwd_cold=cold),
+        "gamma_sweep": sweep, "kv_accounting": accounting,
+        "roofline": roofline, "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 3), "unit": "us/step",
+                "h2d_bytes_per_step": DecodeStep.bytes_of(h_in), "d2h_bytes_per_step": DecodeStep.bytes_of(h_out)},
+        "gpu_launches": launches, "gpu_launches_per_step": launches / args.steps,
+        "clocks": clk, "kernel_source": kernel_source_hash(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """A bounded sample of one windowed-arm decode step for the fp64 oracle: a few query rows of
+    one verify layer at the workload's context, every windowed-draft row of one kv head, and one
+    acceptance.  Inputs are drawn once; ``estimate()`` times the oracle on them and scales each
+    part by the rows the full step has (at a fixed key count the cost per row does not depend on
+    the row)."""
+
+    def __init__(self, w, gamma, window, L, n_q_v, n_layers, rows=None):
+        import numpy as np
+
+        import oracle
+        from synthetic import gen
+
+        self.oracle = oracle
+        self.w, self.gamma, self.window, self.n_q_v, self.n_layers = w, gamma, window, n_q_v, n_layers
+        self.cores = oracle.max_threads()
+        self.rows_n = rows or max(2, self.cores)
+        rng = np.random.default_rng(w.seed)
+        self.Lv = L + n_q_v
+        G, D = w.G, w.D
+        self.kv, self.vv = gen.kv_pair_bf16(rng, (1, 1, self.Lv, D), k_scale=w.k_scale, outlier_p=w.outlier_p)
+        self.qv = gen.normal_bf16(rng, (1, n_q_v, G, D))
+        self.Ld = L + gamma + 1
+        self.kd, self.vd = gen.kv_pair_bf16(rng, (1, 1, self.Ld + gamma, D), k_scale=w.k_scale,
+                                            outlier_p=w.outlier_p)
+        self.qc = gen.normal_bf16(rng, (1, gamma + 1, G, D))
+        self.qf = gen.normal_bf16(rng, (1, 1, G, D))
+        self.logits = gen.uniform_logits(rng, (w.B, n_q_v, w.vocab))
+        self.toks = rng.integers(0, w.vocab, size=(w.B, n_q_v)).astype(np.int32)
+
+    def _time(self, fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    def estimate(self):
+        o, w, g = self.oracle, self.w, self.gamma
+        G = w.G
+        rows = [(0, i % self.n_q_v, (i // self.n_q_v) % G) for i in range(self.rows_n)]
+        t_rows = self._time(lambda: o.attention(self.qv, self.kv, self.vv, [self.Lv], o.MODE_CAUSAL,
+                                                w.sm_scale, rows=rows))
+        scale_v = self.n_q_v * w.Hq * self.n_layers * w.B / self.rows_n
+        t_verify = t_rows * scale_v
+        t_ctx = self._time(lambda: o.attention(self.qc, self.kd, self.vd, [self.Ld], o.MODE_WINDOW,
+                                               w.sm_scale, n_sink=w.n_sink, window=self.window))
+        t_fwd = self._time(lambda: o.attention(self.qf, self.kd, self.vd, [self.Ld + 1], o.MODE_WINDOW,
+                                               w.sm_scale, n_sink=w.n_sink, window=self.window))
+        t_draft = (t_ctx + g * t_fwd) * w.Hkv * w.B
+        t_acc = self._time(lambda: o.accept_greedy(self.logits, self.toks))
+        total = t_verify + t_draft + t_acc
+        return {"value": round(total * 1e6, 1), "unit": "us/step", "cores": self.cores, "kind": "oracle",
+                "sample": f"{self.rows_n} verify query rows at {self.Lv} keys (x{scale_v:.0f}), every "
+                          f"windowed-draft row of one kv head (x{w.Hkv * w.B}), one acceptance",
+                "t_verify_us": round(t_verify * 1e6, 1), "t_draft_windowed_us": round(t_draft * 1e6, 1),
+                "t_accept_us": round(t_acc * 1e6, 1)}
+
+
+def oracle_step_estimate(w, gamma, window, lens, n_q_v, n_layers):
+    return OracleSample(w, gamma, window, int(lens[0]), n_q_v, n_layers).estimate()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from synthetic import configs
+
+    w = configs.BY_NAME[args.workload]
+    window = args.window or w.windows[0]
+    n_q_v = w.tree_nodes or args.gamma + 1
+    lens = [w.L] * w.B if not w.ragged[1] else [(w.ragged[0] + w.ragged[1]) // 2] * w.B
+    sample = OracleSample(w, args.gamma, window, lens[0], n_q_v, w.verify_layers)
+    for _ in range(args.warmup):
+        sample.estimate()
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = sample.estimate()
+        vals.append(r["value"])
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "us/step",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(value / 1e3, 3), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name} (oracle sample per step, scaled)", "gamma": args.gamma,
+                       "window": window},
+            "cpu_baseline": {"value": round(value, 1), "unit": "us/step", "cores": sample.cores,
+                             "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": round(value, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": round(wall, 2)}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

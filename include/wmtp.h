@@ -169,6 +169,10 @@ WMTP_API int accept_greedy(const float* logits, const int32_t* tokens, const int
                   int B, int n_q, int V, int32_t* accepted, int32_t* n_accepted,
                   wmtp_stream_t stream);
 
+/* Number of kernels this library has launched in this process (all devices), for launch
+ * accounting by benchmarks.  Never resets. */
+WMTP_API uint64_t wmtp_launch_count(void);
+
 /* Reads and clears the device status word on the current device (synchronizes `stream`).
  * Returns WMTP_OK, WMTP_ERR_DEVICE_INDEX, or WMTP_ERR_CUDA if the read itself failed. */
 WMTP_API int wmtp_device_status(wmtp_stream_t stream);

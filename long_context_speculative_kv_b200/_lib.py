@@ -38,6 +38,7 @@ _SIGNATURES = {
     "verify_attn": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, SZ, P], I),
     "accept_greedy": ([P, P, P, I, I, I, P, P, P], I),
     "wmtp_device_status": ([P], I),
+    "wmtp_launch_count": ([], ctypes.c_uint64),
 }
 
 

@@ -140,3 +140,8 @@ def accept_greedy(logits, tokens, tree_parent=None, accepted=None, n_accepted=No
 def device_status(stream=None) -> int:
     """Reads and clears the device status word (synchronizes the stream); 0 when clean."""
     return int(lib().wmtp_device_status(_stream(stream)))
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().wmtp_launch_count())

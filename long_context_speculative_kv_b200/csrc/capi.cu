@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "wmtp.h"
@@ -25,6 +26,14 @@ struct DeviceInfo {
 };
 
 std::mutex g_mu;
+std::atomic<unsigned long long> g_launches{0};
+
+// Checks the launch just issued and counts it.
+int launched() {
+    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return WMTP_OK;
+}
 DeviceInfo g_dev[kMaxDevices];
 bool g_dev_done[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -134,10 +143,9 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
         attr_set[dev] = true;
     }
     kern<<<grid, (NMT * NKG + 1) * 32, Lay::kAlloc, st>>>(km, vm, a);
-    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    if (launched() != WMTP_OK) return WMTP_ERR_CUDA;
     lse_merge_kernel<SRC><<<dim3(s.units, s.rows_blk), kD, 0, st>>>(a, grid);
-    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
-    return WMTP_OK;
+    return launched();
 }
 
 template <int SRC>
@@ -266,10 +274,10 @@ int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, cons
         reinterpret_cast<uint4*>(ring_k), reinterpret_cast<uint4*>(ring_v),
         reinterpret_cast<long long*>(ring_len), reinterpret_cast<const uint4*>(k_new),
         reinterpret_cast<const uint4*>(v_new), n_new, Hkv, n_sink, capacity, single);
-    if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+    if (launched() != WMTP_OK) return WMTP_ERR_CUDA;
     if (!single) {
         ring_len_add_kernel<<<(B + 255) / 256, 256, 0, st>>>(reinterpret_cast<long long*>(ring_len), B, n_new);
-        if (cudaGetLastError() != cudaSuccess) return WMTP_ERR_CUDA;
+        if (launched() != WMTP_OK) return WMTP_ERR_CUDA;
     }
     return WMTP_OK;
 }
@@ -331,8 +339,10 @@ int accept_greedy(const float* logits, const int32_t* tokens, const int32_t* tre
     if (rc != WMTP_OK) return rc;
     accept_greedy_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         logits, tokens, tree_parent, n_q, V, accepted, n_accepted);
-    return cudaGetLastError() == cudaSuccess ? WMTP_OK : WMTP_ERR_CUDA;
+    return launched();
 }
+
+uint64_t wmtp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int wmtp_device_status(wmtp_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return WMTP_ERR_CUDA;

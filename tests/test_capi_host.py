@@ -25,7 +25,7 @@ def test_header_declares_the_five_calls_and_helpers():
     names = _declared()
     assert {"ring_kv_append", "draft_attn_window", "draft_attn_full", "verify_attn",
             "accept_greedy", "wmtp_workspace_bytes", "wmtp_status_string",
-            "wmtp_device_status"} == names
+            "wmtp_device_status", "wmtp_launch_count"} == names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -107,3 +107,7 @@ def test_binding_fails_loudly_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libwmtp.so"))
     with pytest.raises(FileNotFoundError):
         _lib.lib()
+
+
+def test_launch_counter_starts_without_launches(lib):
+    assert lib.wmtp_launch_count() == 0      # host-only checks above launched nothing
