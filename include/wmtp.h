@@ -58,7 +58,8 @@ enum wmtp_status {
     WMTP_ERR_CUDA = -5,          /* a CUDA runtime/driver call or launch failed              */
     WMTP_ERR_DEVICE_INDEX = -6,  /* (device status only) a page id was out of range          */
     WMTP_ERR_UNSUPPORTED = -7,   /* the current device is not an sm_100 GPU                  */
-    WMTP_ERR_TIMEOUT = -8        /* (device status only) a bounded wait in a kernel gave up   */
+    WMTP_ERR_TIMEOUT = -8,       /* (device status only) a bounded wait in a kernel gave up   */
+    WMTP_ERR_SCRATCH_LIMIT = -9  /* shape needs more scratch than the built-in array holds    */
 };
 
 /* Limits checked on the host. */
@@ -168,6 +169,32 @@ WMTP_API int verify_attn(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp
 WMTP_API int accept_greedy(const float* logits, const int32_t* tokens, const int32_t* tree_parent,
                   int B, int n_q, int V, int32_t* accepted, int32_t* n_accepted,
                   wmtp_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * draft_attn_window_noalloc -- draft_attn_window without a caller-supplied workspace.
+ * The paper has no counterpart: this entry point exists for callers that cannot allocate device
+ * memory on their decode path -- engines that plan every buffer at start-up and forbid later
+ * allocations, or latency-critical loops that cannot afford cudaMalloc's implicit device
+ * synchronisation -- and so cannot provide the workspace the other attention calls take.
+ *   Arguments, layouts and results are those of draft_attn_window, minus ws / ws_bytes.  The
+ *   split partials go to a scratch array compiled into the library: WMTP_NOALLOC_SCRATCH_BYTES
+ *   (8 MiB) of device memory that every GPU which loads the library holds until the process
+ *   exits.  The call allocates nothing.
+ *   Limit: the shape must fit the scratch, i.e. (number of SMs + B * Hkv * ceil(n_q * Hq / Hkv
+ *   / 64)) partial slots of 33,024 bytes each; on a 148-SM B200 that is B * Hkv * row-blocks
+ *   <= 106.  Larger shapes return WMTP_ERR_SCRATCH_LIMIT and launch nothing.
+ *   The first call on each device looks up the scratch array's device address (with that device
+ *   current); make that first call before any stream capture.
+ *   All calls on one device share the one scratch array and leave their partials in it.  Nothing
+ *   in it has to start at zero (each call writes every partial it reads), but two calls whose
+ *   kernels overlap on the GPU (different streams, no ordering between them) race on it and
+ *   give wrong results: order such calls, or use draft_attn_window with separate workspaces. */
+#define WMTP_NOALLOC_SCRATCH_BYTES (8u << 20)
+WMTP_API int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k,
+                                       const wmtp_bf16* ring_v, const int64_t* ring_len,
+                                       int B, int n_q, int Hq, int Hkv, int D, int n_sink,
+                                       int window, int capacity, float sm_scale,
+                                       wmtp_bf16* out, float* lse, wmtp_stream_t stream);
 
 /* Number of kernels this library has launched in this process (all devices), for launch
  * accounting by benchmarks.  Never resets. */

@@ -12,7 +12,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "wmtp.h")
 STATUS = {
     0: "WMTP_OK", -1: "WMTP_ERR_ARG", -2: "WMTP_ERR_SHAPE", -3: "WMTP_ERR_ALIGN",
     -4: "WMTP_ERR_WORKSPACE", -5: "WMTP_ERR_CUDA", -6: "WMTP_ERR_DEVICE_INDEX",
-    -7: "WMTP_ERR_UNSUPPORTED", -8: "WMTP_ERR_TIMEOUT",
+    -7: "WMTP_ERR_UNSUPPORTED", -8: "WMTP_ERR_TIMEOUT", -9: "WMTP_ERR_SCRATCH_LIMIT",
 }
 
 
@@ -39,6 +39,7 @@ _SIGNATURES = {
     "accept_greedy": ([P, P, P, I, I, I, P, P, P], I),
     "wmtp_device_status": ([P], I),
     "wmtp_launch_count": ([], ctypes.c_uint64),
+    "draft_attn_window_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P], I),
 }
 
 

@@ -83,6 +83,25 @@ def draft_attn_window(q, ring_k, ring_v, ring_len, n_sink: int, window: int, sm_
     return out, lse
 
 
+def draft_attn_window_noalloc(q, ring_k, ring_v, ring_len, n_sink: int, window: int,
+                              sm_scale: float, out=None, lse=None, want_lse: bool = True,
+                              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """draft_attn_window for callers that cannot allocate a workspace: the library's built-in
+    scratch array holds the split partials (one array per GPU, shared by all calls, so calls
+    must not overlap on the GPU)."""
+    _want(q, torch.bfloat16, "q", 4)
+    _want(ring_k, torch.bfloat16, "ring_k", 4)
+    _want(ring_v, torch.bfloat16, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    B, n_q, Hq, D = q.shape
+    _, Hkv, C, _ = ring_k.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_window_noalloc", lib().draft_attn_window_noalloc(
+        _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), B, n_q, Hq, Hkv, D, int(n_sink),
+        int(window), C, float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
 def _paged_checks(q, k_pool, v_pool, page_table, kv_len):
     _want(q, torch.bfloat16, "q", 4)
     _want(k_pool, torch.bfloat16, "k_pool", 4)

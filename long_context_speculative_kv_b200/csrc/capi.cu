@@ -219,6 +219,35 @@ int paged_call(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_p
 }  // namespace
 }  // namespace wmtp
 
+// ---------------------------------------------------------------------------------------------
+// Scratch for draft_attn_window_noalloc: split partials of callers that cannot allocate device
+// memory.  Host code must not use this name as a device address (on the host it is only a
+// stand-in); the address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char wmtp_noalloc_scratch[WMTP_NOALLOC_SCRATCH_BYTES];
+
+namespace wmtp {
+namespace {
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on first use).
+int noalloc_scratch(void** out) {
+    int dev;
+    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, wmtp_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return WMTP_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return WMTP_OK;
+}
+
+}  // namespace
+}  // namespace wmtp
+
 using namespace wmtp;
 
 extern "C" {
@@ -234,6 +263,7 @@ const char* wmtp_status_string(int status) {
         case WMTP_ERR_DEVICE_INDEX: return "device-side index out of range";
         case WMTP_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
         case WMTP_ERR_TIMEOUT: return "device-side wait timed out";
+        case WMTP_ERR_SCRATCH_LIMIT: return "shape exceeds the built-in scratch of the no-alloc call";
         default: return "unknown status";
     }
 }
@@ -340,6 +370,18 @@ int accept_greedy(const float* logits, const int32_t* tokens, const int32_t* tre
     accept_greedy_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         logits, tokens, tree_parent, n_q, V, accepted, n_accepted);
     return launched();
+}
+
+int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,
+                              const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D,
+                              int n_sink, int window, int capacity, float sm_scale, wmtp_bf16* out,
+                              float* lse, wmtp_stream_t stream) {
+    void* scratch = nullptr;
+    int rc = noalloc_scratch(&scratch);
+    if (rc != WMTP_OK) return rc;
+    rc = draft_attn_window(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
+                           sm_scale, out, lse, scratch, WMTP_NOALLOC_SCRATCH_BYTES, stream);
+    return rc == WMTP_ERR_WORKSPACE ? WMTP_ERR_SCRATCH_LIMIT : rc;
 }
 
 uint64_t wmtp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

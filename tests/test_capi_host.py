@@ -25,7 +25,7 @@ def test_header_declares_the_five_calls_and_helpers():
     names = _declared()
     assert {"ring_kv_append", "draft_attn_window", "draft_attn_full", "verify_attn",
             "accept_greedy", "wmtp_workspace_bytes", "wmtp_status_string",
-            "wmtp_device_status", "wmtp_launch_count"} == names
+            "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc"} == names
 
 
 def test_library_exports_every_declared_symbol(lib):
