@@ -41,6 +41,8 @@ def parse():
     p.add_argument("--window", type=int, default=0, help="recent window W (default: the workload's first)")
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--context", type=int, default=0, help="override the committed context (profiling cases)")
+    p.add_argument("--layers", type=int, default=0, help="override the verify layer count (profiling cases)")
     return p.parse_args()
 
 
@@ -154,13 +156,16 @@ def run_gpu(args):
         return float(t.item())
 
     w = configs.BY_NAME[args.workload]
+    if args.context:
+        import dataclasses
+        w = dataclasses.replace(w, L=args.context, ragged=(0, 0), name=f"{w.name}@L{args.context}")
     window = args.window or w.windows[0]
     gammas = sorted(set(w.gammas) | {args.gamma}) if not args.no_sweep else [args.gamma]
     if w.tree_nodes:
         gammas = [args.gamma]
     max_nq = max([w.tree_nodes or (g + 1) for g in gammas])
     shared = workload.shared_inputs(w, device, max_nq_verify=max_nq, max_gamma=max(gammas),
-                                    window=window)
+                                    window=window, n_layers=args.layers or None)
     lens = shared["lens"]
     Lsum = sum(lens)
 
