@@ -180,9 +180,11 @@ WMTP_API int accept_greedy(const float* logits, const int32_t* tokens, const int
  *   split partials go to a scratch array compiled into the library: WMTP_NOALLOC_SCRATCH_BYTES
  *   (8 MiB) of device memory that every GPU which loads the library holds until the process
  *   exits.  The call allocates nothing.
- *   Limit: the shape must fit the scratch, i.e. (number of SMs + B * Hkv * ceil(n_q * Hq / Hkv
- *   / 64)) partial slots of 33,024 bytes each; on a 148-SM B200 that is B * Hkv * row-blocks
- *   <= 106.  Larger shapes return WMTP_ERR_SCRATCH_LIMIT and launch nothing.
+ *   Limit: the shape must fit the scratch: (CTAs the call launches, one or two per SM, plus
+ *   B * Hkv * ceil(n_q * Hq / Hkv / 64)) partial slots of rows * 516 bytes each, rows =
+ *   min(64, n_q * Hq / Hkv).  On a 148-SM B200 a one-query call with 8 query heads per kv head
+ *   fits B * Hkv <= 1884, a 4-query call (32 rows) B * Hkv <= 212.  Larger shapes return
+ *   WMTP_ERR_SCRATCH_LIMIT and launch nothing.
  *   The first call on each device looks up the scratch array's device address (with that device
  *   current); make that first call before any stream capture.
  *   All calls on one device share the one scratch array and leave their partials in it.  Nothing

@@ -41,10 +41,11 @@ struct AttnArgs {
     const __nv_bfloat16* q;      // [B, n_q, Hq, D]
     __nv_bfloat16* out;          // [B, n_q, Hq, D]
     float* lse;                  // [B, n_q, Hq] or null
-    float* ws_o;                 // [slots][64][D]   normalised partial outputs
-    float* ws_lse;               // [slots][64]      base-2 partial log-sum-exp
+    float* ws_o;                 // [slots][rows_blk][D]   normalised partial outputs
+    float* ws_lse;               // [slots][rows_blk]      base-2 partial log-sum-exp
     int B, n_q, Hq, Hkv, G, n_rb;
     int rows_total;              // n_q * G
+    int rows_blk;                // rows per unit (min(64, rows_total)): the workspace slot height
     float scale_log2;            // sm_scale * log2(e)
     const int* tree_parent;      // [B, n_q] or null (chain / causal)
     // paged source
@@ -153,8 +154,8 @@ __device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t base, int row, int 
 }
 
 // ---------------------------------------------------------------------------------------------
-template <int SRC, int NMT, int NKG, int NSTAGE>
-__global__ void __launch_bounds__((NMT * NKG + 1) * 32, 1)
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB>
+__global__ void __launch_bounds__((NMT * NKG + 1) * 32, MINB)
 attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const AttnArgs a) {
     using L = SmemLayout<NMT, NKG, NSTAGE>;
@@ -178,6 +179,13 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+
+    pdl_launch_dependents();
+    if (warp == NWC && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
+    pdl_wait();
 
     // ---- plan: lengths -> tiles per request -> this CTA's tile range ------------------------
     if (warp == NWC) {
@@ -210,8 +218,6 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     if (warp == NWC) {
         // =========================== producer warp =========================================
         if (lane == 0) {
-            prefetch_tensormap(&kmap);
-            prefetch_tensormap(&vmap);
             const uint64_t pol = l2_evict_first_policy();
             int b = 0;
             long long b_start = 0;           // first flat tile of request b
@@ -405,7 +411,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
             }
             // ---- online softmax (base 2) -------------------------------------------------
-            uint32_t pa[NT / 2][4];
+            float m_use[2], alpha[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 float mx = -INFINITY;
@@ -414,16 +420,27 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
                 const float m_new = fmaxf(m_r[r], mx * a.scale_log2);
-                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                const float alpha = fast_exp2(m_r[r] - m_use);
+                m_use[r] = (m_new == -INFINITY) ? 0.f : m_new;
+                alpha[r] = fast_exp2(m_r[r] - m_use[r]);
                 m_r[r] = m_new;
-                l_r[r] *= alpha;
+                l_r[r] *= alpha[r];
+            }
+            // the running maxima rarely move after the first tiles: skip the O rescale when no
+            // row of this warp changed
+            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-                for (int n = 0; n < 16; ++n) { o[n][2 * r] *= alpha; o[n][2 * r + 1] *= alpha; }
+                for (int n = 0; n < 16; ++n) {
+                    o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
+                    o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
+                }
+            }
+            uint32_t pa[NT / 2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
-                    const float p0 = fast_exp2(fmaf(s[n][2 * r], a.scale_log2, -m_use));
-                    const float p1 = fast_exp2(fmaf(s[n][2 * r + 1], a.scale_log2, -m_use));
+                    const float p0 = fast_exp2(fmaf(s[n][2 * r], a.scale_log2, -m_use[r]));
+                    const float p1 = fast_exp2(fmaf(s[n][2 * r + 1], a.scale_log2, -m_use[r]));
                     const uint32_t pk = pack_bf16x2(p0, p1);
                     // the row sum uses the same bf16-rounded weights the PV product uses
                     l_r[r] += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
@@ -525,12 +542,12 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                             op[n * 4 + tig] = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
                         if (a.lse != nullptr && tig == 0) a.lse[orow] = lse2 * kLn2;
                     } else {
-                        float* wo = a.ws_o + ((size_t)slot * kRowsPerBlock + rr) * kD;
+                        float* wo = a.ws_o + ((size_t)slot * a.rows_blk + rr) * kD;
 #pragma unroll
                         for (int n = 0; n < 16; ++n)
                             *reinterpret_cast<float2*>(wo + n * 8 + 2 * tig) =
                                 make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
-                        if (tig == 0) a.ws_lse[(size_t)slot * kRowsPerBlock + rr] = lse2;
+                        if (tig == 0) a.ws_lse[(size_t)slot * a.rows_blk + rr] = lse2;
                     }
                 }
             }
@@ -542,10 +559,15 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 // lse_merge_kernel: combines the split partials of units that span several CTAs, and writes
 // empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block), 128
 // threads (one per head dim).  Partial s has weight 2^(lse_s - max_s lse_s); empty partials have
-// lse = -inf and weight 0.
+// lse = -inf and weight 0.  The partials' LSEs are read by all threads in parallel, then every
+// thread sums its head dim over the partials with independent loads.
+constexpr int kMaxParts = 1024;
+
 template <int SRC>
 __global__ void __launch_bounds__(kD)
 lse_merge_kernel(const AttnArgs a, int P_launch) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int u = blockIdx.x;
     const int rr = blockIdx.y;
     const int rb = u % a.n_rb;
@@ -555,6 +577,8 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     if (R >= a.rows_total) return;
 
     __shared__ long long s_info[3];     // T, unit start, unit tiles
+    __shared__ float s_w[kMaxParts];
+    __shared__ float s_red[kD / 32];
     if (threadIdx.x == 0) {
         long long T = 0, start = 0;
         int nt_u = 0;
@@ -580,18 +604,39 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     const int c_lo = cta_of_tile(start, T, peff);
     const int c_hi = cta_of_tile(start + nt_u - 1, T, peff);
     if (c_lo == c_hi) return;           // finished inside one CTA
+    const int np = c_hi - c_lo + 1;     // <= peff <= P_launch <= kMaxParts (host-checked)
+    const float* lse_base = a.ws_lse + (size_t)(c_lo + u) * a.rows_blk + rr;
     float mx = -INFINITY;
-    for (int c = c_lo; c <= c_hi; ++c)
-        mx = fmaxf(mx, a.ws_lse[(size_t)(c + u) * kRowsPerBlock + rr]);
-    float acc = 0.f, wsum = 0.f;
-    if (mx != -INFINITY) {
-        for (int c = c_lo; c <= c_hi; ++c) {
-            const size_t slot = (size_t)(c + u);
-            const float w = exp2f(a.ws_lse[slot * kRowsPerBlock + rr] - mx);
-            wsum += w;
-            acc += w * a.ws_o[(slot * kRowsPerBlock + rr) * kD + d];
-        }
+    for (int k = d; k < np; k += kD) {
+        const float x = lse_base[(size_t)k * a.rows_blk];
+        s_w[k] = x;
+        mx = fmaxf(mx, x);
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if ((d & 31) == 0) s_red[d >> 5] = mx;
+    __syncthreads();
+    mx = s_red[0];
+#pragma unroll
+    for (int k = 1; k < kD / 32; ++k) mx = fmaxf(mx, s_red[k]);
+    for (int k = d; k < np; k += kD) s_w[k] = (mx == -INFINITY) ? 0.f : exp2f(s_w[k] - mx);
+    __syncthreads();
+    const float* o_base = a.ws_o + ((size_t)(c_lo + u) * a.rows_blk + rr) * kD + d;
+    const size_t kSlotStride = (size_t)a.rows_blk * kD;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, wsum = 0.f;
+    int k = 0;
+    for (; k + 4 <= np; k += 4) {
+        acc0 += s_w[k] * o_base[(size_t)k * kSlotStride];
+        acc1 += s_w[k + 1] * o_base[(size_t)(k + 1) * kSlotStride];
+        acc2 += s_w[k + 2] * o_base[(size_t)(k + 2) * kSlotStride];
+        acc3 += s_w[k + 3] * o_base[(size_t)(k + 3) * kSlotStride];
+        wsum += (s_w[k] + s_w[k + 1]) + (s_w[k + 2] + s_w[k + 3]);
+    }
+    for (; k < np; ++k) {
+        acc0 += s_w[k] * o_base[(size_t)k * kSlotStride];
+        wsum += s_w[k];
+    }
+    const float acc = (acc0 + acc1) + (acc2 + acc3);
     const float res = wsum > 0.f ? acc / wsum : 0.f;
     a.out[orow * kD + d] = __float2bfloat16_rn(res);
     if (a.lse != nullptr && d == 0) a.lse[orow] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;

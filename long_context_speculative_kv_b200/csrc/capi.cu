@@ -5,7 +5,9 @@
 
 #include <cmath>
 #include <cstdlib>
+#include <cstdio>
 #include <cstring>
+#include <utility>
 #include <atomic>
 #include <mutex>
 
@@ -120,20 +122,74 @@ int check_shape(int B, int n_q, int Hq, int Hkv, int D, Shape* s) {
     return WMTP_OK;
 }
 
-// Workspace: [slots][64][128] fp32 partial outputs, then [slots][64] fp32 partial LSEs.
-size_t ws_o_bytes(long long slots) { return (size_t)slots * kRowsPerBlock * kD * sizeof(float); }
-size_t ws_total_bytes(long long slots) {
-    size_t a = (ws_o_bytes(slots) + 255) & ~size_t(255);
-    return a + (size_t)slots * kRowsPerBlock * sizeof(float);
+// Workspace: [slots][rows_blk][128] fp32 partial outputs, then [slots][rows_blk] fp32 partial
+// LSEs (slot = CTA + unit; rows_blk = rows per unit).
+size_t ws_o_bytes(long long slots, int rows_blk) { return (size_t)slots * rows_blk * kD * sizeof(float); }
+size_t ws_total_bytes(long long slots, int rows_blk) {
+    size_t a = (ws_o_bytes(slots, rows_blk) + 255) & ~size_t(255);
+    return a + (size_t)slots * rows_blk * sizeof(float);
 }
 
-constexpr int kStages = 4;
+// ---------------------------------------------------------------------------------------------
+// Launch helpers.  Kernels go out with programmatic stream serialization (PDL) unless
+// WMTP_PDL=0: each kernel lets its successor launch early and waits for its predecessor before
+// touching global memory (see pdl_wait in device_common.cuh).
+bool pdl_enabled() {
+    static bool v = [] {
+        const char* e = std::getenv("WMTP_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return v;
+}
 
-template <int SRC, int NMT, int NKG>
-int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int grid,
+template <typename... KArgs, typename... Args>
+int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+           Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return WMTP_ERR_CUDA;
+    }
+    return launched();
+}
+
+// Attention kernel variants: (key groups NKG, pipeline stages NSTAGE, CTAs per SM MINB) per
+// m-tile count NMT.  Variant 'A' is the default; WMTP_VARIANT_NMT<n>=B|C selects another (for
+// tuning sweeps).  The workspace is sized for the largest grid any variant launches.
+// Measured at 1M keys on B200 (fraction of the measured HBM copy peak; ncu shows the 1-CTA
+// layouts latency-bound with one consumer warp per sub-partition, so two independent CTA
+// pipelines per SM win once rows exceed 16):
+//   rows 16: A (4 key groups, 4 stages, 1 CTA/SM) 1.00
+//   rows 32: A (2, 2, 2 CTAs) 0.97 | (2, 4, 1) 0.81 | (1, 3, 2) 0.82
+//   rows 48: A (1, 2, 2) 0.81 | (1, 3, 2) 0.81 | (2, 4, 1) 0.70
+//   rows 64: A (1, 2, 2) 0.66 | (1, 3, 2) 0.65 | (2, 4, 1) 0.52
+constexpr int kMaxCtasPerSm = 2;
+
+char variant_for(int nmt) {
+    static char v[5] = {0, 0, 0, 0, 0};
+    if (!v[nmt]) {
+        char name[32];
+        std::snprintf(name, sizeof name, "WMTP_VARIANT_NMT%d", nmt);
+        const char* e = std::getenv(name);
+        v[nmt] = (e && (e[0] == 'B' || e[0] == 'C')) ? e[0] : 'A';
+    }
+    return v[nmt];
+}
+
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB>
+int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                   const Shape& s, cudaStream_t st) {
-    using Lay = SmemLayout<NMT, NKG, kStages>;
-    auto kern = attn_split_kernel<SRC, NMT, NKG, kStages>;
+    using Lay = SmemLayout<NMT, NKG, NSTAGE>;
+    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB>;
     static bool attr_set[kMaxDevices] = {};
     int dev;
     if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
@@ -142,22 +198,51 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
             return WMTP_ERR_CUDA;
         attr_set[dev] = true;
     }
-    kern<<<grid, (NMT * NKG + 1) * 32, Lay::kAlloc, st>>>(km, vm, a);
-    if (launched() != WMTP_OK) return WMTP_ERR_CUDA;
-    lse_merge_kernel<SRC><<<dim3(s.units, s.rows_blk), kD, 0, st>>>(a, grid);
-    return launched();
+    const int grid = sm_count * MINB;
+    int rc = launch(kern, dim3(grid), dim3((NMT * NKG + 1) * 32), Lay::kAlloc, st, km, vm, a);
+    if (rc != WMTP_OK) return rc;
+    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
 
 template <int SRC>
-int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int grid,
+int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                 const Shape& s, cudaStream_t st) {
     const int nmt = (s.rows_blk + 15) / 16;
     switch (nmt) {
-        case 1: return launch_attn_t<SRC, 1, 4>(km, vm, a, grid, s, st);
-        case 2: return launch_attn_t<SRC, 2, 2>(km, vm, a, grid, s, st);
-        case 3: return launch_attn_t<SRC, 3, 2>(km, vm, a, grid, s, st);
-        default: return launch_attn_t<SRC, 4, 2>(km, vm, a, grid, s, st);
+        case 1:
+            switch (variant_for(1)) {
+                case 'B': return launch_attn_t<SRC, 1, 4, 2, 2>(km, vm, a, sm_count, s, st);
+                case 'C': return launch_attn_t<SRC, 1, 2, 2, 2>(km, vm, a, sm_count, s, st);
+                default: return launch_attn_t<SRC, 1, 4, 4, 1>(km, vm, a, sm_count, s, st);
+            }
+        case 2:
+            switch (variant_for(2)) {
+                case 'B': return launch_attn_t<SRC, 2, 2, 4, 1>(km, vm, a, sm_count, s, st);
+                case 'C': return launch_attn_t<SRC, 2, 1, 3, 2>(km, vm, a, sm_count, s, st);
+                default: return launch_attn_t<SRC, 2, 2, 2, 2>(km, vm, a, sm_count, s, st);
+            }
+        case 3:
+            switch (variant_for(3)) {
+                case 'B': return launch_attn_t<SRC, 3, 1, 3, 2>(km, vm, a, sm_count, s, st);
+                case 'C': return launch_attn_t<SRC, 3, 2, 4, 1>(km, vm, a, sm_count, s, st);
+                default: return launch_attn_t<SRC, 3, 1, 2, 2>(km, vm, a, sm_count, s, st);
+            }
+        default:
+            switch (variant_for(4)) {
+                case 'B': return launch_attn_t<SRC, 4, 1, 3, 2>(km, vm, a, sm_count, s, st);
+                case 'C': return launch_attn_t<SRC, 4, 2, 4, 1>(km, vm, a, sm_count, s, st);
+                default: return launch_attn_t<SRC, 4, 1, 2, 2>(km, vm, a, sm_count, s, st);
+            }
     }
+}
+
+// CTAs per SM of the variant a call with these rows will use.
+int ctas_per_sm_for(const Shape& s) {
+    const int nmt = (s.rows_blk + 15) / 16;
+    const char v = variant_for(nmt < 4 ? nmt : 4);
+    if (nmt == 1) return v == 'A' ? 1 : 2;
+    if (nmt == 2) return v == 'B' ? 1 : 2;
+    return v == 'C' ? 1 : 2;
 }
 
 // Common front half of the three attention calls.
@@ -169,17 +254,18 @@ int prepare(const Shape& s, const void* q, const void* out, const float* lse, vo
         return WMTP_ERR_ALIGN;
     int rc = device_info(dev);
     if (rc != WMTP_OK) return rc;
-    const long long slots = (long long)dev->sm_count + s.units;
-    if (ws_bytes < ws_total_bytes(slots)) return WMTP_ERR_WORKSPACE;
+    const long long slots = (long long)dev->sm_count * ctas_per_sm_for(s) + s.units;
+    if (ws_bytes < ws_total_bytes(slots, s.rows_blk)) return WMTP_ERR_WORKSPACE;
     std::memset(a, 0, sizeof(*a));
     a->q = reinterpret_cast<const __nv_bfloat16*>(q);
     a->out = reinterpret_cast<__nv_bfloat16*>(const_cast<void*>(out));
     a->lse = const_cast<float*>(lse);
     a->ws_o = reinterpret_cast<float*>(ws);
     a->ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
-                                         ((ws_o_bytes(slots) + 255) & ~size_t(255)));
+                                         ((ws_o_bytes(slots, s.rows_blk) + 255) & ~size_t(255)));
     a->B = s.B; a->n_q = s.n_q; a->Hq = s.Hq; a->Hkv = s.Hkv; a->G = s.G; a->n_rb = s.n_rb;
     a->rows_total = s.rows_total;
+    a->rows_blk = s.rows_blk;
     a->scale_log2 = sm_scale * 1.4426950408889634f;
     a->min_tiles_per_cta = min_tiles_per_cta();
     return WMTP_OK;
@@ -273,7 +359,7 @@ size_t wmtp_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D) {
     if (check_shape(B, n_q, Hq, Hkv, D, &s) != WMTP_OK) return 0;
     DeviceInfo dev;
     if (device_info(&dev) != WMTP_OK) return 0;
-    return ws_total_bytes((long long)dev.sm_count + s.units);
+    return ws_total_bytes((long long)dev.sm_count * kMaxCtasPerSm + s.units, s.rows_blk);
 }
 
 int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, const wmtp_bf16* k_new,
@@ -300,16 +386,13 @@ int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, cons
     if (chunks > max_chunks) chunks = max_chunks;
     if (chunks < 1) chunks = 1;
     const int single = (chunks == 1);
-    ring_append_kernel<<<dim3((unsigned)chunks, B), 256, 0, st>>>(
-        reinterpret_cast<uint4*>(ring_k), reinterpret_cast<uint4*>(ring_v),
-        reinterpret_cast<long long*>(ring_len), reinterpret_cast<const uint4*>(k_new),
-        reinterpret_cast<const uint4*>(v_new), n_new, Hkv, n_sink, capacity, single);
-    if (launched() != WMTP_OK) return WMTP_ERR_CUDA;
-    if (!single) {
-        ring_len_add_kernel<<<(B + 255) / 256, 256, 0, st>>>(reinterpret_cast<long long*>(ring_len), B, n_new);
-        if (launched() != WMTP_OK) return WMTP_ERR_CUDA;
-    }
-    return WMTP_OK;
+    rc = launch(ring_append_kernel, dim3((unsigned)chunks, B), dim3(256), 0, st,
+                reinterpret_cast<uint4*>(ring_k), reinterpret_cast<uint4*>(ring_v),
+                reinterpret_cast<long long*>(ring_len), reinterpret_cast<const uint4*>(k_new),
+                reinterpret_cast<const uint4*>(v_new), n_new, Hkv, n_sink, capacity, single);
+    if (rc != WMTP_OK || single) return rc;
+    return launch(ring_len_add_kernel, dim3((B + 255) / 256), dim3(256), 0, st,
+                  reinterpret_cast<long long*>(ring_len), B, n_new);
 }
 
 int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,
@@ -367,9 +450,8 @@ int accept_greedy(const float* logits, const int32_t* tokens, const int32_t* tre
     DeviceInfo dev;
     int rc = device_info(&dev);
     if (rc != WMTP_OK) return rc;
-    accept_greedy_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        logits, tokens, tree_parent, n_q, V, accepted, n_accepted);
-    return launched();
+    return launch(accept_greedy_kernel, dim3(B), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
+                  logits, tokens, tree_parent, n_q, V, accepted, n_accepted);
 }
 
 int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,

@@ -110,6 +110,16 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library lets the next kernel on the stream
+// launch early (its CTAs then block in pdl_wait) and waits for its own predecessor to finish,
+// with memory visible, before it touches global memory.  Without the launch attribute both are
+// no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------------
 // ldmatrix / mma.sync (bf16 in, fp32 accumulate).
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {

@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(256)
 ring_append_kernel(uint4* __restrict__ ring_k, uint4* __restrict__ ring_v, long long* ring_len,
                    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                    int n_new, int Hkv, int n_sink, int C, int update_len_here) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int b = blockIdx.y;
     const long long L_old = ring_len[b];
     const long long L_new = L_old + n_new;
@@ -54,6 +56,8 @@ ring_append_kernel(uint4* __restrict__ ring_k, uint4* __restrict__ ring_v, long 
 // Length update for appends spread over several CTAs per request (runs after them on the
 // same stream).
 __global__ void ring_len_add_kernel(long long* ring_len, int B, int n_new) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b < B) ring_len[b] += n_new;
 }
@@ -69,6 +73,8 @@ accept_greedy_kernel(const float* __restrict__ logits, const int* __restrict__ t
                      const int* __restrict__ tree_parent, int n_q, int V,
                      int* __restrict__ accepted, int* __restrict__ n_accepted) {
     __shared__ int t_arg[64];
+    pdl_launch_dependents();
+    pdl_wait();
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = warp; i < n_q; i += blockDim.x >> 5) {

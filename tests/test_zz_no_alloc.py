@@ -75,13 +75,15 @@ def test_noalloc_matches_workspace_call_twice_in_a_row():
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():
     lib = _lib.lib()
-    B, Hq, Hkv = 64, 32, 4          # 256 units: more partial slots than the scratch holds
-    q = torch.zeros((B, 1, Hq, D), dtype=torch.bfloat16, device="cuda")
-    ring = torch.zeros((B, Hkv, 4096, D), dtype=torch.bfloat16, device="cuda")
-    rl = torch.full((B,), 4096, dtype=torch.int64, device="cuda")
+    # 64-row units (8 queries x 8 heads per kv head), 16 x 8 of them: with one or two CTAs per SM
+    # that is more than the 254 slots of 64 rows the 8 MiB scratch holds
+    B, n_q, Hq, Hkv, C = 16, 8, 64, 8, 64
+    q = torch.zeros((B, n_q, Hq, D), dtype=torch.bfloat16, device="cuda")
+    ring = torch.zeros((B, Hkv, C, D), dtype=torch.bfloat16, device="cuda")
+    rl = torch.full((B,), C, dtype=torch.int64, device="cuda")
     out = torch.empty_like(q)
     n0 = lib.wmtp_launch_count()
     rc = lib.draft_attn_window_noalloc(q.data_ptr(), ring.data_ptr(), ring.data_ptr(), rl.data_ptr(),
-                                       B, 1, Hq, Hkv, D, 4, 4092, 4096, 0.1, out.data_ptr(), None, None)
+                                       B, n_q, Hq, Hkv, D, 4, C - 4, C, 0.1, out.data_ptr(), None, None)
     assert rc == -9 and "scratch" in _lib.status_string(rc)
     assert lib.wmtp_launch_count() == n0
