@@ -43,6 +43,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--context", type=int, default=0, help="override the committed context (profiling cases)")
     p.add_argument("--layers", type=int, default=0, help="override the verify layer count (profiling cases)")
+    p.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA-graph replays")
     return p.parse_args()
 
 
@@ -208,13 +209,61 @@ def run_gpu(args):
         barrier()
         return e0.elapsed_time(e1), logs, api.launch_count() - n0
 
+    def capture(arm):
+        """One step of `arm` captured as a CUDA graph; returns (graph, library launches in it)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step.run(arm)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        n0 = api.launch_count()
+        with torch.cuda.graph(g):
+            step.run(arm)
+        torch.cuda.synchronize()
+        return g, api.launch_count() - n0
+
+    def timed_graph(g, K, e2e=None):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            if e2e is not None:
+                h_in_, h_out_ = e2e
+                for n, t in h_in_.items():
+                    getattr(step.b, n).copy_(t, non_blocking=True)
+            g.replay()
+            if e2e is not None:
+                for n, t in h_out_.items():
+                    t.copy_(step.b.out[n], non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
+
     props = torch.cuda.get_device_properties(device)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    use_graph = not args.eager
+    if use_graph:
+        g_w, per_step_launches = capture("windowed")
+        g_n, _ = capture("native")
+        for _ in range(2):
+            g_w.replay()
+            g_n.replay()
     clocks = ClockSampler(gpu_id)
     time.sleep(0.3)
-    ms_w, logs_w, launches = timed("windowed", args.steps)
-    ms_n, logs_n, _ = timed("native", args.steps)
+    if use_graph:
+        ms_w = timed_graph(g_w, args.steps)
+        ms_n = timed_graph(g_n, args.steps)
+        launches = per_step_launches * args.steps
+    else:
+        ms_w, _, launches = timed("windowed", args.steps, with_log=False)
+        ms_n, _, _ = timed("native", args.steps, with_log=False)
     clk = clocks.stop()
+    # per-call breakdown from eager launches with CUDA events between calls
+    ms_w_eager, logs_w, _ = timed("windowed", args.steps)
+    ms_n_eager, logs_n, _ = timed("native", args.steps)
     assert api.device_status() == 0
 
     def per_label(logs):
@@ -292,8 +341,13 @@ def run_gpu(args):
     h_in, h_out = step.host_inputs(), step.host_outputs()
     for _ in range(2):
         step.run_e2e("windowed", h_in, h_out)
-    ms_e2e, _, _ = timed("windowed", args.steps, e2e=(h_in, h_out))
+    if use_graph:
+        ms_e2e = timed_graph(g_w, args.steps, e2e=(h_in, h_out))
+    else:
+        ms_e2e, _, _ = timed("windowed", args.steps, e2e=(h_in, h_out))
     e2e_value = max_ranks(ms_e2e) * 1e3 / (args.steps * world)
+    if use_graph:
+        del g_w, g_n
 
     # ---- draft-depth sweep -------------------------------------------------------------
     sweep = {}
@@ -305,8 +359,15 @@ def run_gpu(args):
             for _ in range(2):
                 step.run("windowed")
                 step.run("native")
-            mw, lgw, _ = timed("windowed", Ks)
-            mn, lgn, _ = timed("native", Ks)
+            mw_e, lgw, _ = timed("windowed", Ks)
+            mn_e, lgn, _ = timed("native", Ks)
+            if use_graph:
+                gw, _ = capture("windowed")
+                gn, _ = capture("native")
+                mw, mn = timed_graph(gw, Ks), timed_graph(gn, Ks)
+                del gw, gn
+            else:
+                mw, mn = mw_e, mn_e
             dw, vw, _ = phases(lgw, {"append_ctx", "window_ctx", "append_fwd", "window_fwd"})
             dn, vn, _ = phases(lgn, {"full_ctx", "full_fwd"})
             sweep[str(g)] = {"windowed_us": round(max_ranks(mw) * 1e3 / Ks, 2),
@@ -353,16 +414,18 @@ def run_gpu(args):
            "batch": w.B, "context": lens if w.B <= 8 else Lm,
            "l2": "inputs larger than L2 (each step streams %.1f GiB of KV)" % (sb_w.total * w.B / 2 ** 30),
            "value_is": "windowed-arm us per decode step = max-over-ranks time / (steps x ranks)",
-           "parallelism": f"replicas x{world}"}
+           "parallelism": f"replicas x{world}",
+           "launch_mode": "CUDA graph of one decode step, replayed" if use_graph else "eager launches"}
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "us/step", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1e3, 6),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, random page tables)", "config": cfg,
-        "windowed": {"us_per_step": round(us_w_local, 2), "t_draft_us": round(tdw, 2),
-                     "t_verify_us": round(tvw, 2), "t_accept_us": round(taw, 2)},
-        "native": {"us_per_step": round(us_n_local, 2), "t_draft_us": round(tdn, 2),
-                   "t_verify_us": round(tvn, 2), "t_accept_us": round(tan, 2)},
+        "windowed": {"us_per_step": round(us_w_local, 2), "us_per_step_eager": round(ms_w_eager * 1e3 / args.steps, 2),
+                     "t_draft_us": round(tdw, 2), "t_verify_us": round(tvw, 2), "t_accept_us": round(taw, 2)},
+        "native": {"us_per_step": round(us_n_local, 2), "us_per_step_eager": round(ms_n_eager * 1e3 / args.steps, 2),
+                   "t_draft_us": round(tdn, 2), "t_verify_us": round(tvn, 2), "t_accept_us": round(tan, 2)},
+        "phase_times_from": "eager launches with CUDA events between calls",
         "step_cost_ratio_native_over_windowed": round(ms_n_max / ms_w_max, 4),
         "step_cost_reduction_pct": round(100 * (ms_n_max / ms_w_max - 1), 2),
         "kernels": dict(kernels, draft_attn_window_fwd_cold=cold),

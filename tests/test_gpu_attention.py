@@ -224,3 +224,42 @@ def test_window_covering_context_equals_full():
     assert_attn_close(ow, ref)
     assert_attn_close(of, ref)
     assert np.abs(ow - of).max() <= 1e-2
+
+
+def test_graph_replays_match_eager_calls():
+    """The attention calls captured once in a CUDA graph and replayed (each replay finds the
+    previous replay's partials in the workspace) give the eager results every time."""
+    sc = 128 ** -0.5
+    c = paged_case(9, [7000, 3000], 32, 4, 4)
+    cw = ring_case(10, [9000, 5000], 32, 4, 1, 4, 4092, 4096)
+    B, n_q, Hq, _ = c["q"].shape
+    ws = api.alloc_workspace(B, n_q, Hq, 4)
+    args = (to_dev_bf16(c["q"]), to_dev_bf16(c["kp"]), to_dev_bf16(c["vp"]),
+            torch.from_numpy(c["table"]).cuda(), torch.from_numpy(c["lens"].astype(np.int32)).cuda())
+    qw = to_dev_bf16(cw["q"])
+    ov, lv = torch.empty_like(args[0]), torch.empty(args[0].shape[:3], dtype=torch.float32, device="cuda")
+    ow, lw = torch.empty_like(qw), torch.empty(qw.shape[:3], dtype=torch.float32, device="cuda")
+
+    def calls():
+        api.verify_attn(*args, sc, ws, out=ov, lse=lv)
+        api.draft_attn_window(qw, cw["ring_k"], cw["ring_v"], cw["rlen"], 4, 4092, sc, ws, out=ow, lse=lw)
+
+    calls()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (ov, lv, ow, lw)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        calls()                                   # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        calls()
+    for _ in range(3):
+        for t in (ov, lv, ow, lw):
+            t.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for t, r in zip((ov, lv, ow, lw), ref):
+            assert torch.equal(t, r)
+    assert api.device_status() == 0
