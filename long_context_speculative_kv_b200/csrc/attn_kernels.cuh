@@ -130,6 +130,86 @@ __device__ __forceinline__ int cta_of_tile(long long t, long long T, int P) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Walks a CTA's flat tile range in order and describes each tile: its unit, key positions,
+// valid rows, first/last/whole flags, and the TMA row/block coordinates of its K/V boxes.
+template <int SRC>
+struct TileWalker {
+    int b = 0;
+    long long b_start = 0, per_b = 0;
+
+    __device__ __forceinline__ void init(const AttnArgs& a, const int* plan_tiles) {
+        b = 0;
+        b_start = 0;
+        per_b = (long long)plan_tiles[0] * a.Hkv * a.n_rb;
+    }
+
+    __device__ __forceinline__ void describe(const AttnArgs& a, const int* plan_tiles,
+                                             const int* plan_len, long long t, long long t_begin,
+                                             long long t_end, TileMeta& m, int& ty, int& tz) {
+        while (t >= b_start + per_b) {
+            b_start += per_b;
+            ++b;
+            per_b = (long long)plan_tiles[b] * a.Hkv * a.n_rb;
+        }
+        const int nt_b = plan_tiles[b];
+        const long long off = t - b_start;
+        const int unit_in_b = (int)(off / nt_b);
+        const int tile = (int)(off - (long long)unit_in_b * nt_b);
+        const int h = unit_in_b / a.n_rb;
+        const int rb = unit_in_b - h * a.n_rb;
+        const long long u_start = b_start + (long long)unit_in_b * nt_b;
+        m.b = b; m.h = h; m.rb = rb;
+        m.unit = (b * a.Hkv + h) * a.n_rb + rb;
+        m.L_tot = plan_len[b];
+        m.flags = ((t == t_begin || tile == 0) ? kFirst : 0) |
+                  ((t == t_end - 1 || tile == nt_b - 1) ? kLast : 0) |
+                  ((u_start >= t_begin && u_start + nt_b <= t_end) ? kWhole : 0);
+        if (SRC == kSrcPaged) {
+            const int page = tile < a.max_pages ? a.page_table[(size_t)b * a.max_pages + tile] : -1;
+            m.pos0 = tile * kTileKeys;
+            const int rem = m.L_tot - m.pos0;
+            m.nvalid = rem < kTileKeys ? rem : kTileKeys;
+            if (page < 0 || page >= a.num_pages) {
+                flag_status(kStatusDeviceIndex);
+                m.nvalid = 0;
+            }
+            ty = 0;
+            tz = page * a.Hkv + h;
+        } else {
+            Ranges r = ring_ranges(m.L_tot, a.n_sink, a.window, a.capacity);
+            int tl = tile, k = 0;
+            for (; k < r.n; ++k) {
+                const int ntk = (r.len[k] + kTileKeys - 1) / kTileKeys;
+                if (tl < ntk) break;
+                tl -= ntk;
+            }
+            if (k >= r.n) k = r.n - 1;   // unreachable: tile < request_tiles
+            const int rem = r.len[k] - tl * kTileKeys;
+            m.pos0 = r.pos0[k] + tl * kTileKeys;
+            m.nvalid = rem < kTileKeys ? rem : kTileKeys;
+            ty = r.slot0[k] + tl * kTileKeys;
+            tz = b * a.Hkv + h;
+        }
+    }
+};
+
+// Visibility bitmask of the step's in-call keys for query i: bit j set when the key at
+// position L_tot - n_q + j is visible (chain: j <= i; tree: j on i's root path).
+__device__ __forceinline__ unsigned long long step_visibility(const AttnArgs& a, int b, int i) {
+    if (a.tree_parent != nullptr) {
+        unsigned long long msk = 0ull;
+        int cur = i;
+        for (int k = 0; k < 64 && cur >= 0 && cur < a.n_q; ++k) {
+            msk |= 1ull << cur;
+            const int nxt = a.tree_parent[(size_t)b * a.n_q + cur];
+            cur = (nxt < cur) ? nxt : -1;
+        }
+        return msk;
+    }
+    return (i >= 63) ? ~0ull : ((1ull << (i + 1)) - 1ull);
+}
+
+// ---------------------------------------------------------------------------------------------
 // Shared-memory layout (dynamic; stage buffers 1024-byte aligned for the 128-byte swizzle).
 template <int NMT, int NKG, int NSTAGE>
 struct SmemLayout {
@@ -219,57 +299,13 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         // =========================== producer warp =========================================
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();
-            int b = 0;
-            long long b_start = 0;           // first flat tile of request b
-            long long per_b = (long long)plan_tiles[0] * a.Hkv * a.n_rb;
+            TileWalker<SRC> walk;
+            walk.init(a, plan_tiles);
             uint32_t it = 0;
             for (long long t = t_begin; t < t_end; ++t, ++it) {
-                while (t >= b_start + per_b) {
-                    b_start += per_b;
-                    ++b;
-                    per_b = (long long)plan_tiles[b] * a.Hkv * a.n_rb;
-                }
-                const int nt_b = plan_tiles[b];
-                const long long off = t - b_start;
-                const int unit_in_b = (int)(off / nt_b);
-                const int tile = (int)(off - (long long)unit_in_b * nt_b);
-                const int h = unit_in_b / a.n_rb;
-                const int rb = unit_in_b - h * a.n_rb;
-                const long long u_start = b_start + (long long)unit_in_b * nt_b;
                 TileMeta m;
-                m.b = b; m.h = h; m.rb = rb;
-                m.unit = (b * a.Hkv + h) * a.n_rb + rb;
-                m.L_tot = plan_len[b];
-                m.flags = ((t == t_begin || tile == 0) ? kFirst : 0) |
-                          ((t == t_end - 1 || tile == nt_b - 1) ? kLast : 0) |
-                          ((u_start >= t_begin && u_start + nt_b <= t_end) ? kWhole : 0);
                 int ty = 0, tz = 0;
-                if (SRC == kSrcPaged) {
-                    const int page = tile < a.max_pages ? a.page_table[(size_t)b * a.max_pages + tile] : -1;
-                    m.pos0 = tile * kTileKeys;
-                    const int rem = m.L_tot - m.pos0;
-                    m.nvalid = rem < kTileKeys ? rem : kTileKeys;
-                    if (page < 0 || page >= a.num_pages) {
-                        flag_status(kStatusDeviceIndex);
-                        m.nvalid = 0;
-                    }
-                    ty = 0;
-                    tz = page * a.Hkv + h;
-                } else {
-                    Ranges r = ring_ranges(m.L_tot, a.n_sink, a.window, a.capacity);
-                    int tl = tile, k = 0;
-                    for (; k < r.n; ++k) {
-                        const int ntk = (r.len[k] + kTileKeys - 1) / kTileKeys;
-                        if (tl < ntk) break;
-                        tl -= ntk;
-                    }
-                    if (k >= r.n) k = r.n - 1;   // unreachable: tile < request_tiles
-                    const int rem = r.len[k] - tl * kTileKeys;
-                    m.pos0 = r.pos0[k] + tl * kTileKeys;
-                    m.nvalid = rem < kTileKeys ? rem : kTileKeys;
-                    ty = r.slot0[k] + tl * kTileKeys;
-                    tz = b * a.Hkv + h;
-                }
+                walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
                 const int stage = (int)(it % NSTAGE);
                 const uint32_t phase = (it / NSTAGE) & 1u;
                 if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) break;
@@ -340,18 +376,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
                 row_ok[r] = R < a.rows_total;
                 const int i = row_ok[r] ? R / a.G : 0;
-                unsigned long long msk = 0ull;
-                if (a.tree_parent != nullptr) {
-                    int cur = i;
-                    for (int k = 0; k < 64 && cur >= 0 && cur < a.n_q; ++k) {
-                        msk |= 1ull << cur;
-                        const int nxt = a.tree_parent[(size_t)m.b * a.n_q + cur];
-                        cur = (nxt < cur) ? nxt : -1;
-                    }
-                } else {
-                    msk = (i >= 63) ? ~0ull : ((1ull << (i + 1)) - 1ull);
-                }
-                vis[r] = msk;
+                vis[r] = step_visibility(a, m.b, i);
                 m_r[r] = -INFINITY;
                 l_r[r] = 0.f;
             }

@@ -1,0 +1,468 @@
+// attn_tc_kernels.cuh -- split-KV attention on the 5th-generation tensor cores (tcgen05) for
+// units of up to 64 query rows: the multi-query verify of the Windowed-MTP decode step (Pith
+// verdict on arXiv 2607.21535, pith_extraction.key_machinery: the target verifies gamma + 1
+// positions, or a tree, with full attention), where QK^T and PV are dense [rows x 128] x
+// [128 x 64] contractions per key tile.
+//
+// Same work split, tile walk, masks, partial format and merge as attn_split_kernel; only the
+// math engine differs.  Roles (224 threads, one CTA per SM):
+//   warp 0        K producer: each tile's K (two 64x64 TMA boxes) into an NK-deep ring, and each
+//                 unit's Q rows (one box of n_q x G rows per 64-dim half) into a Q double buffer;
+//   warp 6        V producer: each tile's V into an NV-deep ring.  K is released as soon as
+//                 QK^T has read it and V after PV, so K streams up to NK tiles ahead;
+//   warp 1        owns the tensor memory; lane 0 issues tcgen05.mma:
+//                   S[t % NSB] = Q K^T   (M = 64 rows, N = 64 keys, K = 128, fp32 in TMEM)
+//                   O         += P V     (M = 64, N = 128 dims, K = 64 keys, O stays in TMEM)
+//                 S is issued NSB - 1 tiles ahead of PV, so the tensor core works while the
+//                 softmax warps do; it forwards each tile's description to the softmax warps
+//                 through the S barrier;
+//   warps 2..5    softmax: the M = 64 accumulator keeps row r in TMEM lane 32 (r / 16) + r % 16,
+//                 so warp w sees rows 16 (w % 4) .. + 15; with the 16x32bx2 load both half-warps
+//                 read those rows, lanes 0-15 keys 0-31 and lanes 16-31 keys 32-63 (and O dims
+//                 0-63 / 64-127).  Each thread masks, exponentiates against the row's running
+//                 maximum and writes its half of the P row (bf16, 128-byte swizzled) for the PV
+//                 MMA.  The maximum is only moved when a row's maximum grows by more than 2^8
+//                 (log2 units), and only then is that O row rescaled in TMEM, so the common
+//                 tile touches no O at all.
+// Tensor memory: NSB S buffers of 64 columns, then O (128 columns).  Every wait is bounded; on a
+// timeout all roles stop, the MMA thread waits (bounded) for its own MMAs, all meet at the final
+// barrier and warp 1 frees the tensor memory.
+#pragma once
+
+#include "attn_kernels.cuh"
+#include "tcgen05.cuh"
+
+namespace wmtp {
+
+constexpr int kTcThreads = 224;
+constexpr float kRescaleThreshold = 8.f;   // log2 units
+
+template <int NSB>
+struct TcCols {
+    static constexpr uint32_t kO = NSB * 64;                     // O columns [kO, kO + 128)
+    static constexpr uint32_t kAlloc = (NSB * 64 + 128) <= 256 ? 256 : 512;
+};
+
+template <int NK, int NV, int NSB>
+struct TcLayout {
+    static constexpr int kTileHalf = kHalfBytes;                 // 64 rows x 128 bytes
+    static constexpr int kKOff = 0;                              // NK x [64 keys][128] (2 boxes)
+    static constexpr int kVOff = kKOff + NK * kTileBytes;        // NV x [64 keys][128]
+    static constexpr int kQOff = kVOff + NV * kTileBytes;        // 2 x [64 rows][128]
+    static constexpr int kQBytes = kTileBytes;
+    static constexpr int kPOff = kQOff + 2 * kQBytes;            // NSB x [64 rows][64 keys]
+    static constexpr int kPBytes = kHalfBytes;
+    static constexpr int kBarOff = kPOff + NSB * kPBytes;
+    // kfull[NK] kempty[NK] vfull[NV] vempty[NV] q_full[2] q_free[2] s_full[NSB] s_free[NSB]
+    // p_full[NSB] p_free[NSB] mma_done[1]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 * NSB + 1;
+    static constexpr int kKMetaOff = kBarOff + kNumBars * 8;
+    static constexpr int kSMetaOff = kKMetaOff + NK * (int)sizeof(TileMeta);
+    static constexpr int kPlanOff = kSMetaOff + NSB * (int)sizeof(TileMeta);
+    static constexpr int kPlanBytes = 2 * kMaxBatch * 4;
+    static constexpr int kTmemOff = kPlanOff + kPlanBytes;
+    static constexpr int kTotal = kTmemOff + 16;
+    static constexpr int kAlloc = kTotal + 1024;
+};
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w),
+          "r"(smem_addr(bar))
+        : "memory");
+}
+
+template <int SRC, int NK, int NV, int NSB>
+__global__ void __launch_bounds__(kTcThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+               const __grid_constant__ CUtensorMap qmap, const AttnArgs a) {
+    using L = TcLayout<NK, NV, NSB>;
+    using TCOL = TcCols<NSB>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* kfull = bars;
+    uint64_t* kempty = kfull + NK;
+    uint64_t* vfull = kempty + NK;
+    uint64_t* vempty = vfull + NV;
+    uint64_t* q_full = vempty + NV;
+    uint64_t* q_free = q_full + 2;
+    uint64_t* s_full = q_free + 2;
+    uint64_t* s_free = s_full + NSB;
+    uint64_t* p_full = s_free + NSB;
+    uint64_t* p_free = p_full + NSB;
+    uint64_t* mma_done = p_free + NSB;
+    TileMeta* kmeta = reinterpret_cast<TileMeta*>(smem + L::kKMetaOff);
+    TileMeta* smeta = reinterpret_cast<TileMeta*>(smem + L::kSMetaOff);
+    int* plan_tiles = reinterpret_cast<int*>(smem + L::kPlanOff);
+    int* plan_len = plan_tiles + kMaxBatch;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemOff);
+    __shared__ long long s_range[2];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    pdl_launch_dependents();
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        prefetch_tensormap(&qmap);
+    }
+    pdl_wait();
+
+    // ---- plan (as attn_split_kernel) -----------------------------------------------------
+    if (warp == 0) {
+        for (int b = lane; b < a.B; b += 32) {
+            const int Lb = request_len<SRC>(a, b);
+            plan_len[b] = Lb;
+            plan_tiles[b] = request_tiles<SRC>(a, Lb);
+        }
+        __syncwarp();
+        if (lane == 0) {
+            long long T = 0;
+            for (int b = 0; b < a.B; ++b) T += (long long)plan_tiles[b] * a.Hkv * a.n_rb;
+            const int peff = plan_ctas(T, gridDim.x, a.min_tiles_per_cta);
+            const long long c = blockIdx.x;
+            s_range[0] = c < peff ? cta_begin(c, T, peff) : 0;
+            s_range[1] = c < peff ? cta_begin(c + 1, T, peff) : 0;
+            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], 1); mbar_init(&kempty[k], 1); }
+            for (int k = 0; k < NV; ++k) { mbar_init(&vfull[k], 1); mbar_init(&vempty[k], 1); }
+            for (int k = 0; k < 2; ++k) { mbar_init(&q_full[k], 1); mbar_init(&q_free[k], 1); }
+            for (int k = 0; k < NSB; ++k) {
+                mbar_init(&s_full[k], 2);      // tensor-core completion + the forwarded description
+                mbar_init(&s_free[k], 4);
+                mbar_init(&p_full[k], 4);
+                mbar_init(&p_free[k], 1);
+            }
+            mbar_init(mma_done, 1);
+            fence_barrier_init();
+        }
+    }
+    __syncthreads();
+    const long long t_begin = s_range[0], t_end = s_range[1];
+    if (t_begin >= t_end) return;
+    const uint32_t n = (uint32_t)(t_end - t_begin);
+
+    // ---- tensor memory (whole warp 1) ------------------------------------------------------
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, TCOL::kAlloc);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 || warp == 6) {
+        // =========================== producers ===============================================
+        if (lane == 0) {
+            const bool is_k = (warp == 0);
+            const uint64_t pol = l2_evict_first_policy();
+            TileWalker<SRC> walk;
+            walk.init(a, plan_tiles);
+            uint32_t uidx = 0, it = 0;
+            const uint32_t q_bytes = (uint32_t)a.rows_total * 256u;
+            bool alive = true;
+            for (long long t = t_begin; t < t_end; ++t, ++it) {
+                TileMeta m;
+                int ty = 0, tz = 0;
+                walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
+                if (is_k) {
+                    if (m.flags & kFirst) {
+                        const uint32_t qb = uidx & 1u;
+                        if (!mbar_wait_bounded(&q_free[qb], ((uidx >> 1) & 1u) ^ 1u)) { alive = false; break; }
+                        uint8_t* qdst = smem + L::kQOff + qb * L::kQBytes;
+                        mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+                        tma_load_4d(qdst, &qmap, &q_full[qb], 0, 0, m.h, m.b * a.n_q);
+                        tma_load_4d(qdst + kHalfBytes, &qmap, &q_full[qb], 64, 0, m.h, m.b * a.n_q);
+                        ++uidx;
+                    }
+                    const uint32_t ks = it % NK;
+                    if (!mbar_wait_bounded(&kempty[ks], ((it / NK) & 1u) ^ 1u)) { alive = false; break; }
+                    kmeta[ks] = m;
+                    uint8_t* dst = smem + L::kKOff + ks * kTileBytes;
+                    if (m.nvalid > 0) {
+                        mbar_arrive_expect_tx(&kfull[ks], kTileBytes);
+                        tma_load_3d(dst, &kmap, &kfull[ks], 0, ty, tz, pol);
+                        tma_load_3d(dst + kHalfBytes, &kmap, &kfull[ks], 64, ty, tz, pol);
+                    } else {
+                        mbar_arrive(&kfull[ks]);
+                    }
+                } else {
+                    const uint32_t vs = it % NV;
+                    if (!mbar_wait_bounded(&vempty[vs], ((it / NV) & 1u) ^ 1u)) { alive = false; break; }
+                    uint8_t* dst = smem + L::kVOff + vs * kTileBytes;
+                    if (m.nvalid > 0) {
+                        mbar_arrive_expect_tx(&vfull[vs], kTileBytes);
+                        tma_load_3d(dst, &vmap, &vfull[vs], 0, ty, tz, pol);
+                        tma_load_3d(dst + kHalfBytes, &vmap, &vfull[vs], 64, ty, tz, pol);
+                    } else {
+                        mbar_arrive(&vfull[vs]);
+                    }
+                }
+            }
+            // drain: every issued stage released (no copy still landing at exit)
+            const uint32_t depth = is_k ? NK : NV;
+            uint64_t* empty = is_k ? kempty : vempty;
+            for (uint32_t k = (it > depth ? it - depth : 0); k < it && alive; ++k)
+                if (!mbar_wait_bounded(&empty[k % depth], (k / depth) & 1u)) break;
+        }
+    } else if (warp == 1) {
+        // =========================== MMA issuer ==============================================
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = tc::idesc_bf16_f32(64, 64, false, false);
+            constexpr uint32_t kIdescO = tc::idesc_bf16_f32(64, 128, false, true);
+            // descriptors of the ring bases; a k-step or buffer offset is added as (bytes >> 4)
+            const uint64_t dK = tc::smem_desc(smem_addr(smem + L::kKOff), 16, 1024);
+            const uint64_t dQ = tc::smem_desc(smem_addr(smem + L::kQOff), 16, 1024);
+            const uint64_t dP = tc::smem_desc(smem_addr(smem + L::kPOff), 16, 1024);
+            const uint64_t dV = tc::smem_desc(smem_addr(smem + L::kVOff), 8192, 1024);
+            uint32_t uidx = 0, o_init = 0;
+            bool alive = true;
+            TileMeta mq[NSB];
+            auto issue_s = [&](uint32_t t) -> bool {
+                const uint32_t ks = t % NK;
+                if (!mbar_wait_bounded(&kfull[ks], (t / NK) & 1u)) return false;
+                const TileMeta m = kmeta[ks];
+                if (m.flags & kFirst) {
+                    if (!mbar_wait_bounded(&q_full[uidx & 1u], (uidx >> 1) & 1u)) return false;
+                    ++uidx;
+                }
+                const uint32_t sb = t % NSB;
+                if (!mbar_wait_bounded(&s_free[sb], ((t / NSB) & 1u) ^ 1u)) return false;
+                smeta[sb] = m;
+                mq[sb] = m;
+                tc::fence_after_sync();
+                if (m.nvalid > 0) {
+                    const uint32_t qoff = ((uidx - 1u) & 1u) * (uint32_t)L::kQBytes;
+                    const uint32_t koff = ks * (uint32_t)kTileBytes;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t off = (uint32_t)((j >> 2) * kHalfBytes + (j & 3) * 32);
+                        tc::mma_f16_ss(tmem + sb * 64u, dQ + ((qoff + off) >> 4), dK + ((koff + off) >> 4),
+                                       kIdescS, j > 0);
+                    }
+                }
+                tc::commit(&kempty[ks]);
+                tc::commit(&s_full[sb]);
+                mbar_arrive(&s_full[sb]);
+                if (m.flags & kLast) tc::commit(&q_free[(uidx - 1u) & 1u]);
+                return true;
+            };
+            for (uint32_t t = 0; t + 1 < (uint32_t)NSB && t < n && alive; ++t) alive = issue_s(t);
+            for (uint32_t t = 0; t < n && alive; ++t) {
+                if (t + NSB - 1 < n && !issue_s(t + NSB - 1)) { alive = false; break; }
+                const uint32_t sb = t % NSB, vs = t % NV;
+                const TileMeta m = mq[sb];
+                if (!mbar_wait_bounded(&p_full[sb], (t / NSB) & 1u)) { alive = false; break; }
+                if (!mbar_wait_bounded(&vfull[vs], (t / NV) & 1u)) { alive = false; break; }
+                tc::fence_after_sync();
+                if (m.flags & kFirst) o_init = 0;
+                if (m.nvalid > 0) {
+                    const uint32_t poff = sb * (uint32_t)L::kPBytes;
+                    const uint32_t voff = vs * (uint32_t)kTileBytes;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        tc::mma_f16_ss(tmem + TCOL::kO, dP + ((poff + 32u * j) >> 4),
+                                       dV + ((voff + 2048u * j) >> 4), kIdescO, (o_init | (uint32_t)j) != 0u);
+                    o_init = 1;
+                }
+                tc::commit(&p_free[sb]);
+                tc::commit(&vempty[vs]);
+            }
+            // every MMA of this thread complete before the tensor memory is freed
+            tc::commit(mma_done);
+            mbar_wait_bounded(mma_done, 0);
+        }
+    } else {
+        // =========================== softmax warps ===========================================
+        const int sp = warp & 3;
+        const int half = lane >> 4;
+        const int row = 16 * sp + (lane & 15);
+        const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+        float m_used = -INFINITY, l_part = 0.f;
+        unsigned long long vis = 0ull;
+        bool row_ok = false;
+        int Lpre = 0;
+        bool alive = true;
+        for (uint32_t it = 0; it < n && alive; ++it) {
+            const uint32_t sb = it % NSB;
+            if (!mbar_wait_bounded(&s_full[sb], (it / NSB) & 1u)) { alive = false; break; }
+            tc::fence_after_sync();
+            const TileMeta m = smeta[sb];
+            if (m.flags & kFirst) {
+                Lpre = m.L_tot - a.n_q;
+                const int R = m.rb * kRowsPerBlock + row;
+                row_ok = R < a.rows_total;
+                vis = row_ok ? step_visibility(a, m.b, R / a.G) : 0ull;
+                m_used = -INFINITY;
+                l_part = 0.f;
+            }
+            // ---- this thread's 32 scores from tensor memory ---------------------------------
+            __syncwarp();
+            uint32_t sr[32];
+            tc::ld_16x32bx2_x16<32>(tmem + lane_base + sb * 64u, sr);
+            tc::ld_16x32bx2_x16<32>(tmem + lane_base + sb * 64u + 16u, sr + 16);
+            tc::wait_ld();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sb]);
+            // ---- key mask of this row: valid rows of the tile, prefix keys, visible step keys --
+            uint32_t mk = 0u;
+            if (row_ok && m.nvalid > 0) {
+                if (m.nvalid == kTileKeys && m.pos0 + kTileKeys <= Lpre) {
+                    mk = ~0u;
+                } else {
+                    const int d = Lpre - m.pos0;           // keys [0, d) of the tile are prefix
+                    const unsigned long long valid =
+                        m.nvalid >= 64 ? ~0ull : ((1ull << m.nvalid) - 1ull);
+                    const unsigned long long pre =
+                        d >= 64 ? ~0ull : (d <= 0 ? 0ull : ((1ull << d) - 1ull));
+                    const unsigned long long step =
+                        d >= 64 ? 0ull : (d >= 0 ? (vis << d) : (-d >= 64 ? 0ull : (vis >> (-d))));
+                    mk = (uint32_t)(((pre | step) & valid) >> (32 * half));
+                }
+            }
+            // ---- maximum over the row (both half-warps), running maximum -------------------
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = ((mk >> j) & 1u) ? __uint_as_float(sr[j]) : -INFINITY;
+            float mx8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(fmaxf(x[j], x[j + 8]), fmaxf(x[j + 16], x[j + 24]));
+            float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * a.scale_log2;
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
+                if (m_used != -INFINITY) {
+                    alpha = fast_exp2(m_used - mx);
+                    rescale = true;
+                }
+                m_used = mx;
+                l_part *= alpha;
+            }
+            const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+            uint32_t pk[16];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float p0 = fast_exp2(fmaf(x[2 * j], a.scale_log2, -m_sub));
+                const float p1 = fast_exp2(fmaf(x[2 * j + 1], a.scale_log2, -m_sub));
+                pk[j] = pack_bf16x2(p0, p1);
+                ls[j & 3] += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+            }
+            l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            // ---- P to shared memory (its buffer is free once PV of tile it - NSB is done) -----
+            if (it >= (uint32_t)NSB && !mbar_wait_bounded(&p_free[sb], ((it / NSB) & 1u) ^ 1u)) {
+                alive = false;
+                break;
+            }
+            {
+                uint8_t* prow = smem + L::kPOff + sb * L::kPBytes + row * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int chunk = 4 * half + c;
+                    *reinterpret_cast<uint4*>(prow + ((chunk ^ (row & 7)) << 4)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                }
+            }
+            // V rows past the valid keys may hold anything (NaN tails): zero them before PV
+            if (m.nvalid > 0 && m.nvalid < kTileKeys) {
+                const uint32_t vs = it % NV;
+                if (!mbar_wait_bounded(&vfull[vs], (it / NV) & 1u)) { alive = false; break; }
+                uint8_t* vt = smem + L::kVOff + vs * kTileBytes;
+                const int nrow = kTileKeys - m.nvalid;
+                for (int idx = threadIdx.x - 64; idx < nrow * 16; idx += 128) {
+                    const int r = m.nvalid + idx / 16, c16 = idx % 16;
+                    *reinterpret_cast<uint4*>(vt + (c16 >> 3) * kHalfBytes + r * 128 + (c16 & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            // ---- rare: move this warp's O rows to the new maximum (after PV of tile it - 1) --
+            if (__any_sync(0xffffffffu, rescale)) {
+                const uint32_t pb = (it - 1) % NSB;
+                if (!mbar_wait_bounded(&p_free[pb], ((it - 1) / NSB) & 1u)) { alive = false; break; }
+                tc::fence_after_sync();
+                const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[16];
+                    __syncwarp();
+                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + TCOL::kO + 16u * c, o);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+                    tc::st_16x32bx2_x16<64>(tmem + lane_base + TCOL::kO + 16u * c, o);
+                }
+                tc::wait_st();
+            }
+            fence_proxy_async();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[sb]);
+            // ---- unit end: O rows out of tensor memory ---------------------------------------
+            if (m.flags & kLast) {
+                if (!mbar_wait_bounded(&p_free[sb], (it / NSB) & 1u)) { alive = false; break; }
+                tc::fence_after_sync();
+                const float l_sum = l_part + __shfl_xor_sync(0xffffffffu, l_part, 16);
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const float lse2 = l_sum > 0.f ? m_used + __log2f(l_sum) : -INFINITY;
+                const int R = m.rb * kRowsPerBlock + row;
+                const int i = R / a.G, g = R - (R / a.G) * a.G;
+                const size_t orow = ((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g;
+                const int slot = (int)blockIdx.x + m.unit;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[16];
+                    __syncwarp();
+                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + TCOL::kO + 16u * c, o);
+                    tc::wait_ld();
+                    if (row_ok) {
+                        const int d0 = 64 * half + 16 * c;
+                        float v[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) v[j] = l_sum > 0.f ? __uint_as_float(o[j]) * inv : 0.f;
+                        if (m.flags & kWhole) {
+                            uint4* op = reinterpret_cast<uint4*>(a.out + orow * kD + d0);
+                            op[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                            op[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                                               pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+                        } else {
+                            float4* wo = reinterpret_cast<float4*>(
+                                a.ws_o + ((size_t)slot * a.rows_blk + row) * kD + d0);
+                            wo[0] = make_float4(v[0], v[1], v[2], v[3]);
+                            wo[1] = make_float4(v[4], v[5], v[6], v[7]);
+                            wo[2] = make_float4(v[8], v[9], v[10], v[11]);
+                            wo[3] = make_float4(v[12], v[13], v[14], v[15]);
+                        }
+                    }
+                }
+                if (row_ok && half == 0) {
+                    if (m.flags & kWhole) {
+                        if (a.lse != nullptr) a.lse[orow] = lse2 * kLn2;
+                    } else {
+                        a.ws_lse[(size_t)slot * a.rows_blk + row] = lse2;
+                    }
+                }
+                tc::fence_before_sync();
+            }
+        }
+    }
+
+    // ---- all roles done (or stopped): free the tensor memory --------------------------------
+    __syncwarp();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, TCOL::kAlloc);
+    }
+}
+
+}  // namespace wmtp

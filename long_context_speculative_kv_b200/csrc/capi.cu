@@ -13,6 +13,7 @@
 
 #include "wmtp.h"
 #include "attn_kernels.cuh"
+#include "attn_tc_kernels.cuh"
 #include "ring_accept_kernels.cuh"
 
 namespace wmtp {
@@ -89,6 +90,24 @@ int encode_rows_map(CUtensorMap* map, const void* base, long long rows, long lon
     cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
+}
+
+// Q of a call, [B, n_q, Hq, 128] bf16, viewed per kv head as 4-D (dim, g, h, b * n_q + i) and
+// read in boxes of (64 dims, G heads, 1 kv head, n_q queries): one box lands as the unit's rows
+// i * G + g, 128 bytes each, 128-byte swizzled (the tcgen05 A-operand layout).
+int encode_q_map(CUtensorMap* map, const void* q, int B, int n_q, int Hq, int Hkv) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int rc = encoder(&enc);
+    if (rc != WMTP_OK) return rc;
+    const int G = Hq / Hkv;
+    cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)G, (cuuint64_t)Hkv, (cuuint64_t)B * n_q};
+    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)G * kD * 2, (cuuint64_t)Hq * kD * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)n_q};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
@@ -204,9 +223,71 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
     return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
 
+// Which units run on the tcgen05 kernel: WMTP_TC=on for units of 33..64 rows, WMTP_TC=all for
+// every unit of at most 64 rows; default off (the mma.sync layouts measure faster so far).
+int tc_mode() {
+    static int v = [] {
+        const char* e = std::getenv("WMTP_TC");
+        if (e && e[0] == 'a') return 2;
+        if (e && e[0] == 'o' && e[1] == 'n') return 1;
+        return 0;
+    }();
+    return v;
+}
+
+bool use_tc(const Shape& s) {
+    if (s.rows_total > kRowsPerBlock) return false;
+    const int mode = tc_mode();
+    return mode == 2 || (mode == 1 && s.rows_blk > 32);
+}
+
+// tcgen05 kernel variants (K ring, V ring, S/P buffers), one CTA per SM: A = (6, 4, 3),
+// B = (4, 3, 2).  WMTP_TC_VARIANT=B selects B (sweeps).
+char tc_variant() {
+    static char v = [] {
+        const char* e = std::getenv("WMTP_TC_VARIANT");
+        return (e && e[0] == 'B') ? 'B' : 'A';
+    }();
+    return v;
+}
+
+int tc_ctas_per_sm() { return 1; }
+
+template <int SRC, int NK, int NV, int NSB>
+int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
+                     int sm_count, const Shape& s, cudaStream_t st) {
+    using Lay = TcLayout<NK, NV, NSB>;
+    auto kern = attn_tc_kernel<SRC, NK, NV, NSB>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev;
+    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess)
+            return WMTP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    CUtensorMap qm;
+    int rc = encode_q_map(&qm, q, s.B, s.n_q, s.Hq, s.Hkv);
+    if (rc != WMTP_OK) return rc;
+    const int grid = sm_count;
+    rc = launch(kern, dim3(grid), dim3(kTcThreads), Lay::kAlloc, st, km, vm, qm, a);
+    if (rc != WMTP_OK) return rc;
+    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
+}
+
+template <int SRC>
+int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
+                   int sm_count, const Shape& s, cudaStream_t st) {
+    switch (tc_variant()) {
+        case 'B': return launch_attn_tc_t<SRC, 4, 3, 2>(km, vm, q, a, sm_count, s, st);
+        default: return launch_attn_tc_t<SRC, 6, 4, 3>(km, vm, q, a, sm_count, s, st);
+    }
+}
+
 template <int SRC>
 int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                 const Shape& s, cudaStream_t st) {
+    if (use_tc(s)) return launch_attn_tc<SRC>(km, vm, a.q, a, sm_count, s, st);
     const int nmt = (s.rows_blk + 15) / 16;
     switch (nmt) {
         case 1:
@@ -238,6 +319,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
 
 // CTAs per SM of the variant a call with these rows will use.
 int ctas_per_sm_for(const Shape& s) {
+    if (use_tc(s)) return tc_ctas_per_sm();
     const int nmt = (s.rows_blk + 15) / 16;
     const char v = variant_for(nmt < 4 ? nmt : 4);
     if (nmt == 1) return v == 'A' ? 1 : 2;

@@ -263,3 +263,26 @@ def test_graph_replays_match_eager_calls():
         for t, r in zip((ov, lv, ow, lw), ref):
             assert torch.equal(t, r)
     assert api.device_status() == 0
+
+
+@pytest.mark.parametrize("n_q,Hq,Hkv,tree", [(8, 32, 4, False), (8, 32, 4, True), (6, 64, 8, False),
+                                             (4, 32, 4, False), (1, 32, 4, False)])
+def test_rising_scores_move_the_running_maximum(n_q, Hq, Hkv, tree):
+    """Scores that grow along the context move every row's running maximum many times (the
+    kernels' rescale paths, which random N(0, 1) inputs rarely reach)."""
+    sc = 128 ** -0.5
+    rng = np.random.default_rng(21)
+    L = 5000 + n_q
+    rise = np.linspace(0.0, 20.0, L, dtype=np.float32)[None, None, :, None]
+    q = gen.bf16_bits(0.2 + 0.05 * rng.standard_normal((1, n_q, Hq, D), dtype=np.float32))
+    k = gen.bf16_bits(rise + 0.3 * rng.standard_normal((1, Hkv, L, D), dtype=np.float32))
+    v = gen.normal_bf16(rng, (1, Hkv, L, D))
+    table = gen.page_table(rng, [L], 64)
+    c = dict(q=q, k=k, v=v, table=table, lens=np.array([L], np.int64),
+             kp=gen.paginate(k, [L], table, 64), vp=gen.paginate(v, [L], table, 64))
+    parent = gen.draft_tree(np.random.default_rng(5), n_q)[None] if tree else None
+    out, lse = run_paged(c, "verify", sc, tree=parent)
+    mode = oracle.MODE_TREE if tree else oracle.MODE_CAUSAL
+    ref, ref_lse = oracle.attention(q, k, v, c["lens"], mode, sc, tree_parent=parent)
+    assert_attn_close(out, ref, "rising scores")
+    assert_lse_close(lse, ref_lse)
