@@ -5,17 +5,18 @@
 // [128 x 64] contractions per key tile.
 //
 // Same work split, tile walk, masks, partial format and merge as attn_split_kernel; only the
-// math engine differs.  Roles (224 threads, one CTA per SM):
+// math engine differs.  Roles (256 threads, one CTA per SM):
 //   warp 0        K producer: each tile's K (two 64x64 TMA boxes) into an NK-deep ring, and each
 //                 unit's Q rows (one box of n_q x G rows per 64-dim half) into a Q double buffer;
 //   warp 6        V producer: each tile's V into an NV-deep ring.  K is released as soon as
 //                 QK^T has read it and V after PV, so K streams up to NK tiles ahead;
-//   warp 1        owns the tensor memory; lane 0 issues tcgen05.mma:
-//                   S[t % NSB] = Q K^T   (M = 64 rows, N = 64 keys, K = 128, fp32 in TMEM)
-//                   O         += P V     (M = 64, N = 128 dims, K = 64 keys, O stays in TMEM)
-//                 S is issued NSB - 1 tiles ahead of PV, so the tensor core works while the
-//                 softmax warps do; it forwards each tile's description to the softmax warps
+//   warp 1        owns the tensor memory; lane 0 issues S[t % NSB] = Q K^T (tcgen05.mma,
+//                 M = 64 rows, N = 64 keys, K = 128, fp32 in TMEM) as soon as a K tile and an S
+//                 buffer are ready, and forwards each tile's description to the softmax warps
 //                 through the S barrier;
+//   warp 7        lane 0 issues O += P V (M = 64, N = 128 dims, K = 64 keys; O stays in TMEM)
+//                 once the softmax warps have written P(t).  Two issuers keep the tensor core's
+//                 queue fed while the other waits;
 //   warps 2..5    softmax: the M = 64 accumulator keeps row r in TMEM lane 32 (r / 16) + r % 16,
 //                 so warp w sees rows 16 (w % 4) .. + 15; with the 16x32bx2 load both half-warps
 //                 read those rows, lanes 0-15 keys 0-31 and lanes 16-31 keys 32-63 (and O dims
@@ -25,7 +26,7 @@
 //                 (log2 units), and only then is that O row rescaled in TMEM, so the common
 //                 tile touches no O at all.
 // Tensor memory: NSB S buffers of 64 columns, then O (128 columns).  Every wait is bounded; on a
-// timeout all roles stop, the MMA thread waits (bounded) for its own MMAs, all meet at the final
+// timeout all roles stop, each MMA issuer waits (bounded) for its own MMAs, all meet at the final
 // barrier and warp 1 frees the tensor memory.
 #pragma once
 
@@ -34,7 +35,7 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 224;
+constexpr int kTcThreads = 256;
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
 template <int NSB>
@@ -54,11 +55,12 @@ struct TcLayout {
     static constexpr int kPBytes = kHalfBytes;
     static constexpr int kBarOff = kPOff + NSB * kPBytes;
     // kfull[NK] kempty[NK] vfull[NV] vempty[NV] q_full[2] q_free[2] s_full[NSB] s_free[NSB]
-    // p_full[NSB] p_free[NSB] mma_done[1]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 * NSB + 1;
+    // p_full[NSB] p_free[NSB] mma_done[2]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 * NSB + 2;
     static constexpr int kKMetaOff = kBarOff + kNumBars * 8;
     static constexpr int kSMetaOff = kKMetaOff + NK * (int)sizeof(TileMeta);
-    static constexpr int kPlanOff = kSMetaOff + NSB * (int)sizeof(TileMeta);
+    static constexpr int kPMetaOff = kSMetaOff + NSB * (int)sizeof(TileMeta);
+    static constexpr int kPlanOff = kPMetaOff + NSB * (int)sizeof(TileMeta);
     static constexpr int kPlanBytes = 2 * kMaxBatch * 4;
     static constexpr int kTmemOff = kPlanOff + kPlanBytes;
     static constexpr int kTotal = kTmemOff + 16;
@@ -97,6 +99,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     uint64_t* mma_done = p_free + NSB;
     TileMeta* kmeta = reinterpret_cast<TileMeta*>(smem + L::kKMetaOff);
     TileMeta* smeta = reinterpret_cast<TileMeta*>(smem + L::kSMetaOff);
+    TileMeta* pmeta = reinterpret_cast<TileMeta*>(smem + L::kPMetaOff);
     int* plan_tiles = reinterpret_cast<int*>(smem + L::kPlanOff);
     int* plan_len = plan_tiles + kMaxBatch;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemOff);
@@ -137,7 +140,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 mbar_init(&p_full[k], 4);
                 mbar_init(&p_free[k], 1);
             }
-            mbar_init(mma_done, 1);
+            mbar_init(&mma_done[0], 1);
+            mbar_init(&mma_done[1], 1);
             fence_barrier_init();
         }
     }
@@ -211,30 +215,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 if (!mbar_wait_bounded(&empty[k % depth], (k / depth) & 1u)) break;
         }
     } else if (warp == 1) {
-        // =========================== MMA issuer ==============================================
+        // =========================== S issuer (QK^T) =========================================
         if (lane == 0) {
             constexpr uint32_t kIdescS = tc::idesc_bf16_f32(64, 64, false, false);
-            constexpr uint32_t kIdescO = tc::idesc_bf16_f32(64, 128, false, true);
             // descriptors of the ring bases; a k-step or buffer offset is added as (bytes >> 4)
             const uint64_t dK = tc::smem_desc(smem_addr(smem + L::kKOff), 16, 1024);
             const uint64_t dQ = tc::smem_desc(smem_addr(smem + L::kQOff), 16, 1024);
-            const uint64_t dP = tc::smem_desc(smem_addr(smem + L::kPOff), 16, 1024);
-            const uint64_t dV = tc::smem_desc(smem_addr(smem + L::kVOff), 8192, 1024);
-            uint32_t uidx = 0, o_init = 0;
-            bool alive = true;
-            TileMeta mq[NSB];
-            auto issue_s = [&](uint32_t t) -> bool {
+            uint32_t uidx = 0;
+            for (uint32_t t = 0; t < n; ++t) {
                 const uint32_t ks = t % NK;
-                if (!mbar_wait_bounded(&kfull[ks], (t / NK) & 1u)) return false;
+                if (!mbar_wait_bounded(&kfull[ks], (t / NK) & 1u)) break;
                 const TileMeta m = kmeta[ks];
                 if (m.flags & kFirst) {
-                    if (!mbar_wait_bounded(&q_full[uidx & 1u], (uidx >> 1) & 1u)) return false;
+                    if (!mbar_wait_bounded(&q_full[uidx & 1u], (uidx >> 1) & 1u)) break;
                     ++uidx;
                 }
                 const uint32_t sb = t % NSB;
-                if (!mbar_wait_bounded(&s_free[sb], ((t / NSB) & 1u) ^ 1u)) return false;
+                if (!mbar_wait_bounded(&s_free[sb], ((t / NSB) & 1u) ^ 1u)) break;
                 smeta[sb] = m;
-                mq[sb] = m;
                 tc::fence_after_sync();
                 if (m.nvalid > 0) {
                     const uint32_t qoff = ((uidx - 1u) & 1u) * (uint32_t)L::kQBytes;
@@ -250,15 +248,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 tc::commit(&s_full[sb]);
                 mbar_arrive(&s_full[sb]);
                 if (m.flags & kLast) tc::commit(&q_free[(uidx - 1u) & 1u]);
-                return true;
-            };
-            for (uint32_t t = 0; t + 1 < (uint32_t)NSB && t < n && alive; ++t) alive = issue_s(t);
-            for (uint32_t t = 0; t < n && alive; ++t) {
-                if (t + NSB - 1 < n && !issue_s(t + NSB - 1)) { alive = false; break; }
+            }
+            // every MMA of this thread complete before the tensor memory is freed
+            tc::commit(&mma_done[0]);
+            mbar_wait_bounded(&mma_done[0], 0);
+        }
+    } else if (warp == 7) {
+        // =========================== PV issuer ===============================================
+        if (lane == 0) {
+            constexpr uint32_t kIdescO = tc::idesc_bf16_f32(64, 128, false, true);
+            const uint64_t dP = tc::smem_desc(smem_addr(smem + L::kPOff), 16, 1024);
+            const uint64_t dV = tc::smem_desc(smem_addr(smem + L::kVOff), 8192, 1024);
+            uint32_t o_init = 0;
+            for (uint32_t t = 0; t < n; ++t) {
                 const uint32_t sb = t % NSB, vs = t % NV;
-                const TileMeta m = mq[sb];
-                if (!mbar_wait_bounded(&p_full[sb], (t / NSB) & 1u)) { alive = false; break; }
-                if (!mbar_wait_bounded(&vfull[vs], (t / NV) & 1u)) { alive = false; break; }
+                // the softmax warps have written P(t) (and read this tile's description) by now
+                if (!mbar_wait_bounded(&p_full[sb], (t / NSB) & 1u)) break;
+                const TileMeta m = pmeta[sb];
+                if (!mbar_wait_bounded(&vfull[vs], (t / NV) & 1u)) break;
                 tc::fence_after_sync();
                 if (m.flags & kFirst) o_init = 0;
                 if (m.nvalid > 0) {
@@ -273,9 +280,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 tc::commit(&p_free[sb]);
                 tc::commit(&vempty[vs]);
             }
-            // every MMA of this thread complete before the tensor memory is freed
-            tc::commit(mma_done);
-            mbar_wait_bounded(mma_done, 0);
+            tc::commit(&mma_done[1]);
+            mbar_wait_bounded(&mma_done[1], 0);
         }
     } else {
         // =========================== softmax warps ===========================================
@@ -401,6 +407,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 }
                 tc::wait_st();
             }
+            if (warp == 2 && lane == 0) pmeta[sb] = m;   // the PV issuer's copy of the description
             fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();

@@ -223,14 +223,16 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
     return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
 
-// Which units run on the tcgen05 kernel: WMTP_TC=on for units of 33..64 rows, WMTP_TC=all for
-// every unit of at most 64 rows; default off (the mma.sync layouts measure faster so far).
+// Which units run on the tcgen05 kernel: by default units of 33..64 rows (at 1M keys on B200:
+// 48 rows 392 us vs 405 us for the best mma.sync layout, 64 rows 403 us vs 498 us, where the
+// legacy tensor pipe limits mma.sync); WMTP_TC=0 turns it off, WMTP_TC=all uses it for every
+// unit of at most 64 rows (tuning sweeps).
 int tc_mode() {
     static int v = [] {
         const char* e = std::getenv("WMTP_TC");
         if (e && e[0] == 'a') return 2;
-        if (e && e[0] == 'o' && e[1] == 'n') return 1;
-        return 0;
+        if (e && e[0] == '0') return 0;
+        return 1;
     }();
     return v;
 }
