@@ -378,6 +378,54 @@ def run_gpu(args):
                 100 * (sweep[str(g)]["native_us"] / sweep[str(g)]["windowed_us"] - 1), 2)
         step = base_step
 
+    # ---- context sweep and linear fit of the draft terms (the Table 6 analogue) ------------
+    ctx_sweep = None
+    if not args.no_sweep and w.B == 1 and not w.tree_nodes:
+        Ls = [x for x in (1 << 16, 1 << 17, 1 << 18, 1 << 19, 1 << 20) if x <= lens[0]]
+        if len(Ls) >= 3:
+            Kc = max(5, args.steps // 10)
+            pts = []
+            for Lx in Ls:
+                st = DecodeStep(StepBuffers(**workload.step_inputs(w, shared, args.gamma, device,
+                                                                   lens=[Lx])), args.gamma)
+                step, keep = st, step
+                for _ in range(2):
+                    step.run("windowed")
+                    step.run("native")
+                _, lgw, _ = timed("windowed", Kc)
+                _, lgn, _ = timed("native", Kc)
+                if use_graph:
+                    gw, _ = capture("windowed")
+                    gn, _ = capture("native")
+                    mw, mn = timed_graph(gw, Kc), timed_graph(gn, Kc)
+                    del gw, gn
+                else:
+                    mw, _, _ = timed("windowed", Kc, with_log=False)
+                    mn, _, _ = timed("native", Kc, with_log=False)
+                step = keep
+                lw_, ln_ = per_label(lgw), per_label(lgn)
+                fwd_w = [a + b for a, b in zip(lw_["append_fwd"], lw_["window_fwd"])]
+                ctx_w = [a + b for a, b in zip(lw_["append_ctx"], lw_["window_ctx"])]
+                pts.append({"L": Lx,
+                            "t_fwd_draft_windowed_us": round(statistics.mean(fwd_w) * 1e3, 3),
+                            "t_fwd_draft_native_us": round(statistics.mean(ln_["full_fwd"]) * 1e3, 3),
+                            "t_ctx_draft_windowed_us": round(statistics.mean(ctx_w) * 1e3, 3),
+                            "t_ctx_draft_native_us": round(statistics.mean(ln_["full_ctx"]) * 1e3, 3),
+                            "step_windowed_us": round(max_ranks(mw) * 1e3 / Kc, 2),
+                            "step_native_us": round(max_ranks(mn) * 1e3 / Kc, 2)})
+                del st
+            fits = {}
+            xs = [p_["L"] for p_ in pts]
+            for key in ("t_fwd_draft_windowed_us", "t_fwd_draft_native_us", "t_ctx_draft_windowed_us",
+                        "t_ctx_draft_native_us", "step_windowed_us", "step_native_us"):
+                m, c, r2 = acc.linear_fit(xs, [p_[key] for p_ in pts])
+                fits[key[:-3]] = {"slope_us_per_1k_tokens": round(m * 1e3, 5),
+                                  "intercept_us": round(c, 3), "r2": round(r2, 5)}
+            sn, sw = fits["step_native"]["slope_us_per_1k_tokens"], fits["step_windowed"]["slope_us_per_1k_tokens"]
+            ctx_sweep = {"points": pts, "fits": fits, "gamma": args.gamma,
+                         "step_slope_reduction_pct": round(100 * (1 - sw / sn), 2) if sn > 0 else None,
+                         "timing": "step: CUDA-graph replay; per-call terms: eager launches with events"}
+
     # ---- KV accounting -------------------------------------------------------------------
     sb_w = acc.step_bytes(int(statistics.mean(lens)), args.gamma, n_q_v, w.Hkv, w.D, n_layers,
                           w.n_sink, window, windowed=True)
@@ -429,7 +477,7 @@ def run_gpu(args):
         "step_cost_ratio_native_over_windowed": round(ms_n_max / ms_w_max, 4),
         "step_cost_reduction_pct": round(100 * (ms_n_max / ms_w_max - 1), 2),
         "kernels": dict(kernels, draft_attn_window_fwd_cold=cold),
-        "gamma_sweep": sweep, "kv_accounting": accounting,
+        "gamma_sweep": sweep, "context_sweep": ctx_sweep, "kv_accounting": accounting,
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 3), "unit": "us/step",
                 "h2d_bytes_per_step": DecodeStep.bytes_of(h_in), "d2h_bytes_per_step": DecodeStep.bytes_of(h_out)},

@@ -80,3 +80,28 @@ def step_bytes(L: int, gamma: int, n_q_verify: int, Hkv: int, D: int, n_layers: 
         ctx = draft_full_bytes(base, Hkv, D)
         fwd = draft_full_bytes(base + gamma, Hkv, D)
     return StepBytes(ctx, fwd, n_layers * verify_layer_bytes(L, n_q_verify, Hkv, D), gamma)
+
+
+def linear_fit(x, y):
+    """Ordinary least squares y = intercept + slope * x, with the coefficient of determination.
+
+    The cost identity's draft terms are fitted against context length this way (Pith verdict on
+    arXiv 2607.21535, referee_report.minor_comments on App. B, Table 6: fitted slopes and
+    intercepts with R^2): a full-context draft forward grows with L, a windowed one should not.
+    Returns (slope, intercept, r2); r2 is 1.0 when y is constant and exactly fitted.
+    """
+    n = len(x)
+    if n != len(y) or n < 2:
+        raise ValueError("linear_fit needs two or more (x, y) pairs")
+    mx = sum(x) / n
+    my = sum(y) / n
+    sxx = sum((a - mx) ** 2 for a in x)
+    if sxx == 0:
+        raise ValueError("linear_fit needs two distinct x values")
+    sxy = sum((a - mx) * (b - my) for a, b in zip(x, y))
+    slope = sxy / sxx
+    intercept = my - slope * mx
+    ss_res = sum((b - (intercept + slope * a)) ** 2 for a, b in zip(x, y))
+    ss_tot = sum((b - my) ** 2 for b in y)
+    r2 = 1.0 - ss_res / ss_tot if ss_tot > 0 else 1.0
+    return slope, intercept, r2

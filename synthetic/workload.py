@@ -43,11 +43,19 @@ def shared_inputs(w, device, seed: Optional[int] = None, max_nq_verify: int = 8,
     return out
 
 
-def step_inputs(w, shared: Dict, gamma: int, device, seed: Optional[int] = None) -> Dict:
-    """Keyword arguments for StepBuffers at draft depth gamma."""
+def step_inputs(w, shared: Dict, gamma: int, device, seed: Optional[int] = None,
+                lens: Optional[Sequence[int]] = None) -> Dict:
+    """Keyword arguments for StepBuffers at draft depth gamma.  ``lens`` runs the step at shorter
+    committed contexts than the buffers were built for (the context sweep): the caches and page
+    tables are reused, only the lengths change."""
     seed = (w.seed if seed is None else seed) * 1000 + gamma
     g = tg.generator(seed, device)
-    lens = shared["lens"]
+    if lens is None:
+        lens = shared["lens"]
+    else:
+        lens = [int(x) for x in lens]
+        if any(a > b for a, b in zip(lens, shared["lens"])) or len(lens) != len(shared["lens"]):
+            raise ValueError("step_inputs: lens must not exceed the built contexts")
     B, Hq, Hkv, D = w.B, w.Hq, w.Hkv, w.D
     n_q = w.tree_nodes if w.tree_nodes else gamma + 1
     n_layers = len(shared["k_pools"])
@@ -71,7 +79,7 @@ def step_inputs(w, shared: Dict, gamma: int, device, seed: Optional[int] = None)
     )
     if "ring_k" in shared:
         kw.update(ring_k=shared["ring_k"], ring_v=shared["ring_v"],
-                  ring_len=shared["ring_len0"].clone())
+                  ring_len=torch.tensor(lens, dtype=torch.int64, device=device))
     if "k_draft" in shared:
         kw.update(k_draft=shared["k_draft"], v_draft=shared["v_draft"], table_d=shared["table_d"],
                   kv_len_ctx=torch.tensor([L + gamma + 1 for L in lens], dtype=torch.int32, device=device),
