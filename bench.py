@@ -41,6 +41,9 @@ def parse():
     p.add_argument("--window", type=int, default=0, help="recent window W (default: the workload's first)")
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-loop", action="store_true", help="skip the decode-loop measurement")
+    p.add_argument("--agree", type=float, default=0.8,
+                   help="decode loop: probability a synthetic draft proposal is the target's token")
     p.add_argument("--context", type=int, default=0, help="override the committed context (profiling cases)")
     p.add_argument("--layers", type=int, default=0, help="override the verify layer count (profiling cases)")
     p.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA-graph replays")
@@ -135,6 +138,7 @@ def run_gpu(args):
 
     from long_context_speculative_kv_b200 import accounting as acc
     from long_context_speculative_kv_b200 import api
+    from long_context_speculative_kv_b200.loop import DecodeLoop, LoopState
     from long_context_speculative_kv_b200.step import CallLog, DecodeStep, StepBuffers
     from synthetic import configs, workload
 
@@ -165,8 +169,11 @@ def run_gpu(args):
     if w.tree_nodes:
         gammas = [args.gamma]
     max_nq = max([w.tree_nodes or (g + 1) for g in gammas])
+    do_loop = not args.no_loop and not w.tree_nodes
+    loop_extra = 24                                   # untimed loop steps per arm (warm-up, breakdown)
+    slack = (max(gammas) + 1) * (args.steps + args.warmup + loop_extra) if do_loop else 0
     shared = workload.shared_inputs(w, device, max_nq_verify=max_nq, max_gamma=max(gammas),
-                                    window=window, n_layers=args.layers or None)
+                                    window=window, n_layers=args.layers or None, slack=slack)
     lens = shared["lens"]
     Lsum = sum(lens)
 
@@ -426,6 +433,74 @@ def run_gpu(args):
                          "step_slope_reduction_pct": round(100 * (1 - sw / sn), 2) if sn > 0 else None,
                          "timing": "step: CUDA-graph replay; per-call terms: eager launches with events"}
 
+    # ---- decode loop: real acceptance from the synthetic heads, rollback, graph per step -------
+    loop_res = None
+    if do_loop:
+        agree24 = int(round(args.agree * (1 << 24)))
+        T0 = [L + 1 for L in lens]
+
+        def make_loop(arm_seed):
+            kw = workload.step_inputs(w, shared, args.gamma, device, seed=w.seed + 17 * arm_seed)
+            gl = torch.Generator(device=device)
+            gl.manual_seed(w.seed + 99)
+            hist = torch.randint(0, w.vocab, (w.B, max(T0) + slack), generator=gl, device=device,
+                                 dtype=torch.int32)
+            state = LoopState.start(hist, T0, args.gamma)
+            C = w.n_sink + window + args.gamma
+            rk = torch.empty((w.B, w.Hkv, C, w.D), dtype=torch.bfloat16, device=device).normal_(generator=gl)
+            rv = torch.empty_like(rk).normal_(generator=gl)
+            kw.update(ring_k=rk, ring_v=rv, ring_len=torch.zeros(w.B, dtype=torch.int64, device=device),
+                      kv_len_v=state.verify_len)
+            return DecodeLoop(StepBuffers(**kw), args.gamma, state, w.vocab, w.seed + 1000, w.seed + 2000, agree24)
+
+        loop_res = {"agree": args.agree, "gamma": args.gamma,
+                    "step": "ring append at the committed position (rollback) + window ctx pass, gamma "
+                            "forwards, synthetic draft proposals, verify x layers, synthetic target "
+                            "logits, accept_greedy, spec_commit; one CUDA graph per step"}
+        for arm in ("windowed", "native"):
+            lp = make_loop(0 if arm == "windowed" else 1)
+            for _ in range(2):
+                lp.step(arm)
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                lp.step(arm)
+            torch.cuda.current_stream().wait_stream(side)
+            gl_ = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gl_):
+                lp.step(arm)
+            for _ in range(args.warmup):
+                gl_.replay()
+            torch.cuda.synchronize()
+            t_before = lp.s.n_tokens.clone()
+            ms = timed_graph(gl_, args.steps)
+            committed = int((lp.s.n_tokens - t_before).sum().item())
+            del gl_
+            logs = []
+            for _ in range(8):
+                lg = CallLog()
+                lp.step(arm, lg)
+                logs.append(lg)
+            torch.cuda.synchronize()
+            assert api.device_status() == 0
+            d = per_label(logs)
+            draft_labels = ("append_ctx", "window_ctx", "append_fwd", "window_fwd", "full_ctx", "full_fwd")
+            ms_max = max_ranks(ms)
+            loop_res[arm] = {
+                "us_per_step": round(ms_max * 1e3 / args.steps, 2),
+                "tokens_committed": committed,
+                "mean_accepted_per_step": round(committed / (args.steps * w.B), 4),
+                "us_per_token": round(ms_max * 1e3 / max(1, committed), 2),
+                "t_draft_us": round(sum(statistics.mean(d[k]) * len(d[k]) / len(logs) for k in draft_labels if k in d) * 1e3, 2),
+                "t_ctx_draft_us": round(sum(statistics.mean(d[k]) for k in ("append_ctx", "window_ctx", "full_ctx") if k in d) * 1e3, 2),
+                "t_verify_us": round(statistics.mean(d["verify"]) * len(d["verify"]) / len(logs) * 1e3, 2),
+                "t_heads_accept_commit_us": round(sum(statistics.mean(d[k]) for k in ("propose", "target_logits", "accept", "commit")) * 1e3, 2),
+            }
+            del lp
+        loop_res["step_cost_reduction_pct"] = round(
+            100 * (loop_res["native"]["us_per_step"] / loop_res["windowed"]["us_per_step"] - 1), 2)
+        loop_res["per_token_speedup"] = round(loop_res["native"]["us_per_token"] / loop_res["windowed"]["us_per_token"], 4)
+
     # ---- KV accounting -------------------------------------------------------------------
     sb_w = acc.step_bytes(int(statistics.mean(lens)), args.gamma, n_q_v, w.Hkv, w.D, n_layers,
                           w.n_sink, window, windowed=True)
@@ -477,7 +552,8 @@ def run_gpu(args):
         "step_cost_ratio_native_over_windowed": round(ms_n_max / ms_w_max, 4),
         "step_cost_reduction_pct": round(100 * (ms_n_max / ms_w_max - 1), 2),
         "kernels": dict(kernels, draft_attn_window_fwd_cold=cold),
-        "gamma_sweep": sweep, "context_sweep": ctx_sweep, "kv_accounting": accounting,
+        "gamma_sweep": sweep, "context_sweep": ctx_sweep, "decode_loop": loop_res,
+        "kv_accounting": accounting,
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 3), "unit": "us/step",
                 "h2d_bytes_per_step": DecodeStep.bytes_of(h_in), "d2h_bytes_per_step": DecodeStep.bytes_of(h_out)},

@@ -7,7 +7,9 @@ import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libwmtp.so")
-HEADER = os.path.join(os.path.dirname(PKG), "include", "wmtp.h")
+INCLUDE = os.path.join(os.path.dirname(PKG), "include")
+HEADER = os.path.join(INCLUDE, "wmtp.h")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 STATUS = {
     0: "WMTP_OK", -1: "WMTP_ERR_ARG", -2: "WMTP_ERR_SHAPE", -3: "WMTP_ERR_ALIGN",
@@ -28,6 +30,9 @@ P = ctypes.c_void_p
 I = ctypes.c_int
 F = ctypes.c_float
 SZ = ctypes.c_size_t
+I64 = ctypes.c_int64
+U64 = ctypes.c_uint64
+U32 = ctypes.c_uint32
 
 _SIGNATURES = {
     "wmtp_status_string": ([I], ctypes.c_char_p),
@@ -40,6 +45,10 @@ _SIGNATURES = {
     "wmtp_device_status": ([P], I),
     "wmtp_launch_count": ([], ctypes.c_uint64),
     "draft_attn_window_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P], I),
+    "ring_kv_append_at": ([P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
+    "spec_commit": ([P, P, I, I, P, I64, P, P, P, P, I, P, I, P], I),
+    "wmtp_synth_draft_tokens": ([P, P, I, I64, I, I, U64, U64, U32, P, P], I),
+    "wmtp_synth_target_logits": ([P, P, I, I64, P, P, I, I, U64, P, P], I),
 }
 
 

@@ -164,3 +164,80 @@ def device_status(stream=None) -> int:
 def launch_count() -> int:
     """Kernels the library has launched in this process so far."""
     return int(lib().wmtp_launch_count())
+
+
+# ----------------------------------------------------------------------------- decode loop
+def ring_kv_append_at(ring_k, ring_v, ring_len, k_new, v_new, pos, n_new, n_sink: int,
+                      stream=None) -> None:
+    """Request b writes rows [0, n_new[b]) of k_new/v_new [B, n_max, Hkv, 128] at draft positions
+    pos[b] ..; ring_len[b] becomes pos[b] + n_new[b] (rolling back anything past it)."""
+    _want(ring_k, torch.bfloat16, "ring_k", 4)
+    _want(ring_v, torch.bfloat16, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    _want(k_new, torch.bfloat16, "k_new", 4)
+    _want(v_new, torch.bfloat16, "v_new", 4)
+    _want(pos, torch.int64, "pos", 1)
+    _want(n_new, torch.int32, "n_new", 1)
+    B, Hkv, C, D = ring_k.shape
+    n_max = k_new.shape[1]
+    if k_new.shape != (B, n_max, Hkv, D) or v_new.shape != k_new.shape or ring_v.shape != ring_k.shape:
+        raise ValueError("ring_kv_append_at: inconsistent shapes")
+    check("ring_kv_append_at", lib().ring_kv_append_at(
+        _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(n_new),
+        B, n_max, Hkv, D, int(n_sink), C, _stream(stream)))
+
+
+def spec_commit(accepted, n_accepted, history, n_tokens, append_pos, n_append, verify_len=None,
+                n_q_verify: int = 0, draft_len=None, stream=None) -> None:
+    """Commits accept_greedy's output into the loop state (see wmtp_loop.h)."""
+    _want(accepted, torch.int32, "accepted", 2)
+    _want(n_accepted, torch.int32, "n_accepted", 1)
+    _want(history, torch.int32, "history", 2)
+    _want(n_tokens, torch.int64, "n_tokens", 1)
+    _want(append_pos, torch.int64, "append_pos", 1)
+    _want(n_append, torch.int32, "n_append", 1)
+    if verify_len is not None:
+        _want(verify_len, torch.int32, "verify_len", 1)
+    n_draft = 0
+    if draft_len is not None:
+        _want(draft_len, torch.int32, "draft_len", 2)
+        n_draft = draft_len.shape[0]
+    B, n_q = accepted.shape
+    check("spec_commit", lib().spec_commit(
+        _ptr(accepted), _ptr(n_accepted), B, n_q, _ptr(history), history.shape[1], _ptr(n_tokens),
+        _ptr(append_pos), _ptr(n_append), _ptr(verify_len), int(n_q_verify), _ptr(draft_len), n_draft,
+        _stream(stream)))
+
+
+def synth_draft_tokens(history, n_tokens, gamma: int, vocab: int, target_seed: int, draft_seed: int,
+                       agree24: int, tokens=None, stream=None):
+    """Synthetic draft head: tokens [B, gamma + 1] (last committed token, then gamma proposals)."""
+    _want(history, torch.int32, "history", 2)
+    _want(n_tokens, torch.int64, "n_tokens", 1)
+    B = history.shape[0]
+    if tokens is None:
+        tokens = torch.empty((B, gamma + 1), dtype=torch.int32, device=history.device)
+    _want(tokens, torch.int32, "tokens", 2)
+    check("wmtp_synth_draft_tokens", lib().wmtp_synth_draft_tokens(
+        _ptr(history), _ptr(n_tokens), B, history.shape[1], int(gamma), int(vocab),
+        int(target_seed) & 0xFFFFFFFFFFFFFFFF, int(draft_seed) & 0xFFFFFFFFFFFFFFFF, int(agree24),
+        _ptr(tokens), _stream(stream)))
+    return tokens
+
+
+def synth_target_logits(history, n_tokens, tokens, vocab: int, target_seed: int, tree_parent=None,
+                        logits=None, stream=None):
+    """Synthetic target head: logits [B, n_q, vocab] of the verify nodes ``tokens`` [B, n_q]."""
+    _want(history, torch.int32, "history", 2)
+    _want(n_tokens, torch.int64, "n_tokens", 1)
+    _want(tokens, torch.int32, "tokens", 2)
+    if tree_parent is not None:
+        _want(tree_parent, torch.int32, "tree_parent", 2)
+    B, n_q = tokens.shape
+    if logits is None:
+        logits = torch.empty((B, n_q, vocab), dtype=torch.float32, device=tokens.device)
+    _want(logits, torch.float32, "logits", 3)
+    check("wmtp_synth_target_logits", lib().wmtp_synth_target_logits(
+        _ptr(history), _ptr(n_tokens), B, history.shape[1], _ptr(tokens), _ptr(tree_parent), n_q,
+        int(vocab), int(target_seed) & 0xFFFFFFFFFFFFFFFF, _ptr(logits), _stream(stream)))
+    return logits

@@ -12,9 +12,12 @@
 #include <mutex>
 
 #include "wmtp.h"
+#include "wmtp_loop.h"
 #include "attn_kernels.cuh"
 #include "attn_tc_kernels.cuh"
 #include "ring_accept_kernels.cuh"
+#include "loop_kernels.cuh"
+#include "synth_kernels.cuh"
 
 namespace wmtp {
 
@@ -548,6 +551,95 @@ int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k, const
     rc = draft_attn_window(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
                            sm_scale, out, lse, scratch, WMTP_NOALLOC_SCRATCH_BYTES, stream);
     return rc == WMTP_ERR_WORKSPACE ? WMTP_ERR_SCRATCH_LIMIT : rc;
+}
+
+int ring_kv_append_at(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, const wmtp_bf16* k_new,
+                      const wmtp_bf16* v_new, const int64_t* pos, const int32_t* n_new, int B, int n_max,
+                      int Hkv, int D, int n_sink, int capacity, wmtp_stream_t stream) {
+    if (ring_k == nullptr || ring_v == nullptr || ring_len == nullptr || k_new == nullptr ||
+        v_new == nullptr || pos == nullptr || n_new == nullptr)
+        return WMTP_ERR_ARG;
+    if (reinterpret_cast<const void*>(pos) == reinterpret_cast<const void*>(ring_len)) return WMTP_ERR_ARG;
+    if (B < 1 || n_max < 1 || Hkv < 1 || n_sink < 0 || capacity <= n_sink) return WMTP_ERR_ARG;
+    if (D != WMTP_HEAD_DIM) return WMTP_ERR_SHAPE;
+    if (B > 65535) return WMTP_ERR_SHAPE;
+    if (!aligned(ring_k, 16) || !aligned(ring_v, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+        !aligned(ring_len, 8) || !aligned(pos, 8) || !aligned(n_new, 4))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    const long long surv = (long long)(n_max < capacity ? n_max : capacity);
+    long long chunks = (surv * Hkv * 16 + 256 * 4 - 1) / (256 * 4);
+    const long long max_chunks = (long long)dev.sm_count * 8;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    return launch(ring_append_at_kernel, dim3((unsigned)chunks, B), dim3(256), 0,
+                  reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<uint4*>(ring_k),
+                  reinterpret_cast<uint4*>(ring_v), reinterpret_cast<long long*>(ring_len),
+                  reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new),
+                  reinterpret_cast<const long long*>(pos), reinterpret_cast<const int*>(n_new), n_max,
+                  Hkv, n_sink, capacity);
+}
+
+int spec_commit(const int32_t* accepted, const int32_t* n_accepted, int B, int n_q, int32_t* history,
+                int64_t max_tokens, int64_t* n_tokens, int64_t* append_pos, int32_t* n_append,
+                int32_t* verify_len, int n_q_verify, int32_t* draft_len, int n_draft,
+                wmtp_stream_t stream) {
+    if (accepted == nullptr || n_accepted == nullptr || history == nullptr || n_tokens == nullptr ||
+        append_pos == nullptr || n_append == nullptr)
+        return WMTP_ERR_ARG;
+    if (B < 1 || n_q < 1 || n_q > WMTP_MAX_QUERIES || max_tokens < 1 || n_draft < 0 || n_q_verify < 0)
+        return WMTP_ERR_ARG;
+    if (max_tokens + (int64_t)n_q_verify + (int64_t)n_draft >= ((int64_t)1 << 31)) return WMTP_ERR_ARG;
+    if (!aligned(accepted, 4) || !aligned(n_accepted, 4) || !aligned(history, 4) ||
+        !aligned(n_tokens, 8) || !aligned(append_pos, 8) || !aligned(n_append, 4) ||
+        (verify_len && !aligned(verify_len, 4)) || (draft_len && !aligned(draft_len, 4)))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    return launch(spec_commit_kernel, dim3((B + 127) / 128), dim3(128), 0,
+                  reinterpret_cast<cudaStream_t>(stream), accepted, n_accepted, B, n_q, history,
+                  (long long)max_tokens, reinterpret_cast<long long*>(n_tokens),
+                  reinterpret_cast<long long*>(append_pos), n_append, verify_len, n_q_verify,
+                  draft_len, n_draft);
+}
+
+int wmtp_synth_draft_tokens(const int32_t* history, const int64_t* n_tokens, int B, int64_t max_tokens,
+                            int gamma, int V, uint64_t target_seed, uint64_t draft_seed, uint32_t agree24,
+                            int32_t* tokens, wmtp_stream_t stream) {
+    if (history == nullptr || n_tokens == nullptr || tokens == nullptr) return WMTP_ERR_ARG;
+    if (B < 1 || V < 2 || gamma < 0 || gamma + 1 > WMTP_MAX_QUERIES || max_tokens < 1 ||
+        agree24 > (1u << 24))
+        return WMTP_ERR_ARG;
+    if (!aligned(history, 4) || !aligned(n_tokens, 8) || !aligned(tokens, 4)) return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    return launch(synth::draft_tokens_kernel, dim3(B), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
+                  history, reinterpret_cast<const long long*>(n_tokens), (long long)max_tokens, gamma, V,
+                  (unsigned long long)target_seed, (unsigned long long)draft_seed, (unsigned int)agree24,
+                  tokens);
+}
+
+int wmtp_synth_target_logits(const int32_t* history, const int64_t* n_tokens, int B, int64_t max_tokens,
+                             const int32_t* tokens, const int32_t* tree_parent, int n_q, int V,
+                             uint64_t target_seed, float* logits, wmtp_stream_t stream) {
+    if (history == nullptr || n_tokens == nullptr || tokens == nullptr || logits == nullptr)
+        return WMTP_ERR_ARG;
+    if (B < 1 || B > 65535 || V < 2 || n_q < 1 || n_q > WMTP_MAX_QUERIES || max_tokens < 1)
+        return WMTP_ERR_ARG;
+    if (!aligned(history, 4) || !aligned(n_tokens, 8) || !aligned(tokens, 4) || !aligned(logits, 4) ||
+        (tree_parent && !aligned(tree_parent, 4)))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    return launch(synth::target_logits_kernel, dim3(n_q, B), dim3(256), 0,
+                  reinterpret_cast<cudaStream_t>(stream), history,
+                  reinterpret_cast<const long long*>(n_tokens), (long long)max_tokens, tokens, tree_parent,
+                  n_q, V, (unsigned long long)target_seed, logits);
 }
 
 uint64_t wmtp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

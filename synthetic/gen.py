@@ -183,3 +183,21 @@ def draft_proposals(policy: str, rng: np.random.Generator, target_next, gamma: i
         else:
             out.append((t + 1 + int(rng.integers(vocab - 1))) % vocab)
     return out
+
+
+def hash_draft_tokens(target_seed: int, draft_seed: int, prefix: Sequence[int], gamma: int,
+                      vocab: int, agree24: int) -> List[int]:
+    """gamma chained proposals of the counter-based synthetic draft: proposal j extends the
+    prefix (and proposals 0..j-1) by the synthetic target's greedy token when
+    (z >> 40) < agree24, z = mix(mix(draft_seed ^ length) ^ (uint32)(last + 1)), and by
+    (greedy + 1 + mix(z) mod (vocab - 1)) mod vocab otherwise (mix = splitmix64)."""
+    out: List[int] = []
+    for _ in range(gamma):
+        path = list(prefix) + out
+        greedy = int(np.argmax(target_logits(target_seed, path, vocab)))
+        z = splitmix64(splitmix64(np.uint64(draft_seed & 0xFFFFFFFFFFFFFFFF) ^ np.uint64(len(path)))
+                       ^ np.uint64((int(path[-1]) + 1) & 0xFFFFFFFF))
+        agree = int(z >> np.uint64(40)) < agree24
+        r = int(splitmix64(z)) % (vocab - 1)
+        out.append(greedy if agree else (greedy + 1 + r) % vocab)
+    return out

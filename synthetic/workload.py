@@ -14,14 +14,16 @@ from . import torch_gen as tg
 
 def shared_inputs(w, device, seed: Optional[int] = None, max_nq_verify: int = 8,
                   max_gamma: int = 7, window: Optional[int] = None, n_layers: Optional[int] = None,
-                  arms: Sequence[str] = ("windowed", "native")) -> Dict:
+                  arms: Sequence[str] = ("windowed", "native"), slack: int = 0) -> Dict:
+    """``slack`` extra positions in the verify layers' caches and the native draft cache, for a
+    decode loop that advances the committed context."""
     seed = w.seed if seed is None else seed
     g = tg.generator(seed, device)
     lens = tg.contexts(w, seed)
     P, D = w.page_size, w.D
     n_layers = w.verify_layers if n_layers is None else n_layers
     window = w.windows[0] if window is None else window
-    lens_v = [L + max_nq_verify for L in lens]
+    lens_v = [L + max_nq_verify + slack for L in lens]
     table_v, npg_v = tg.page_table(lens_v, P, seed + 1)
     k_pools, v_pools = [], []
     for _ in range(n_layers):
@@ -36,7 +38,7 @@ def shared_inputs(w, device, seed: Optional[int] = None, max_nq_verify: int = 8,
         out.update(ring_k=ring_k, ring_v=ring_v,
                    ring_len0=torch.tensor(lens, dtype=torch.int64, device=device))
     if "native" in arms:
-        lens_d = [L + 2 * max_gamma + 1 for L in lens]
+        lens_d = [L + 2 * max_gamma + 1 + slack for L in lens]
         table_d, npg_d = tg.page_table(lens_d, P, seed + 2)
         kd, vd = tg.paged_kv(lens_d, w.Hkv, D, P, g, device, table_d, npg_d, w.k_scale, w.outlier_p)
         out.update(k_draft=kd, v_draft=vd, table_d=torch.from_numpy(table_d).to(device))

@@ -64,3 +64,22 @@ def speculative_greedy(seed: int, prompt: List[int], n_tokens: int, vocab: int, 
         counts.append(n)
         seq.extend(int(t) for t in acc[0, :n])
     return seq[len(prompt):len(prompt) + n_tokens], counts
+
+
+def hash_draft_loop(target_seed: int, draft_seed: int, prompt: List[int], steps: int, vocab: int,
+                    gamma: int, agree24: int, accept: Callable):
+    """The decode loop of the device library on the CPU: per step the counter-based synthetic
+    draft proposes gamma chained tokens, the synthetic target scores the gamma + 1 nodes, and
+    ``accept`` (chain) decides.  Returns (committed sequence after the prompt, accepted counts)."""
+    seq = list(prompt)
+    counts = []
+    for _ in range(steps):
+        props = gen.hash_draft_tokens(target_seed, draft_seed, seq, gamma, vocab, agree24)
+        nodes = [seq[-1]] + props
+        paths = [seq + props[:i] for i in range(gamma + 1)]
+        logits = np.stack([gen.target_logits(target_seed, p, vocab) for p in paths])[None]
+        acc, n_acc = accept(logits, np.asarray(nodes, dtype=np.int32)[None], None)
+        n = int(n_acc[0])
+        counts.append(n)
+        seq.extend(int(t) for t in acc[0, :n])
+    return seq[len(prompt):], counts

@@ -16,16 +16,22 @@ def lib():
     return _lib.lib()
 
 
+def _headers_src():
+    return "\n".join(open(h).read() for h in _lib.HEADERS)
+
+
 def _declared():
-    src = open(_lib.HEADER).read()
-    return set(re.findall(r"^WMTP_API\s+[\w\s\*]*?\b(\w+)\s*\(", src, re.M))
+    return set(re.findall(r"^WMTP_API\s+[\w\s\*]*?\b(\w+)\s*\(", _headers_src(), re.M))
 
 
 def test_header_declares_the_five_calls_and_helpers():
     names = _declared()
     assert {"ring_kv_append", "draft_attn_window", "draft_attn_full", "verify_attn",
             "accept_greedy", "wmtp_workspace_bytes", "wmtp_status_string",
-            "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc"} == names
+            "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc",
+            "ring_kv_append_at", "spec_commit", "wmtp_synth_draft_tokens",
+            "wmtp_synth_target_logits"} == names
+    assert set(_lib._SIGNATURES) == names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -45,7 +51,7 @@ def test_status_strings(lib):
 
 
 def test_binding_signatures_match_header_arity():
-    src = open(_lib.HEADER).read()
+    src = _headers_src()
     for name, (args, _) in _lib._SIGNATURES.items():
         m = re.search(r"^WMTP_API\s+[\w\s\*]*?\b" + name + r"\s*\(([^)]*)\)", src, re.S | re.M)
         assert m, name
@@ -93,6 +99,33 @@ def test_accept_host_checks(lib):
     assert a(GOOD, GOOD, None, 1, 65, 1024, GOOD, GOOD, None) == -1
     assert a(GOOD, GOOD, None, 1, 4, 0, GOOD, GOOD, None) == -1
     assert a(ctypes.c_void_p(0x10002), GOOD, None, 1, 4, 1024, GOOD, GOOD, None) == -3
+
+
+def test_loop_host_checks(lib):
+    r = lib.ring_kv_append_at
+    # (rk, rv, rlen, k_new, v_new, pos, n_new, B, n_max, Hkv, D, s, C, stream)
+    G2 = ctypes.c_void_p(0x20000)
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, G2, None, 1, 4, 2, 128, 4, 256, None) == -1   # null n_new
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, G2, 1, 4, 2, 128, 4, 256, None) == -1   # pos aliases ring_len
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, G2, G2, 1, 0, 2, 128, 4, 256, None) == -1     # n_max < 1
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, G2, G2, 1, 4, 2, 64, 4, 256, None) == -2      # D != 128
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, ctypes.c_void_p(0x20004), G2, 1, 4, 2, 128, 4, 256, None) == -3
+    c = lib.spec_commit
+    # (acc, n_acc, B, n_q, hist, max_tokens, n_tokens, append_pos, n_append, vlen, nqv, dlen, nd, s)
+    assert c(GOOD, GOOD, 1, 4, None, 100, GOOD, GOOD, GOOD, None, 4, None, 0, None) == -1
+    assert c(GOOD, GOOD, 1, 65, GOOD, 100, GOOD, GOOD, GOOD, None, 4, None, 0, None) == -1
+    assert c(GOOD, GOOD, 1, 4, GOOD, (1 << 31) - 2, GOOD, GOOD, GOOD, None, 4, None, 0, None) == -1
+    assert c(GOOD, GOOD, 1, 4, GOOD, 100, ctypes.c_void_p(0x10004), GOOD, GOOD, None, 4, None, 0, None) == -3
+    d = lib.wmtp_synth_draft_tokens
+    # (hist, n_tokens, B, max_tokens, gamma, V, tseed, dseed, agree24, tokens, s)
+    assert d(GOOD, GOOD, 1, 100, 3, 1, 1, 2, 1 << 23, GOOD, None) == -1                  # V < 2
+    assert d(GOOD, GOOD, 1, 100, 64, 1024, 1, 2, 1 << 23, GOOD, None) == -1              # gamma + 1 > 64
+    assert d(GOOD, GOOD, 1, 100, 3, 1024, 1, 2, (1 << 24) + 1, GOOD, None) == -1         # agree24 > 2^24
+    t = lib.wmtp_synth_target_logits
+    # (hist, n_tokens, B, max_tokens, tokens, parent, n_q, V, tseed, logits, s)
+    assert t(GOOD, GOOD, 1, 100, GOOD, None, 0, 1024, 1, GOOD, None) == -1
+    assert t(GOOD, GOOD, 1, 100, GOOD, None, 4, 1024, 1, None, None) == -1
+    assert t(GOOD, GOOD, 1, 100, GOOD, ctypes.c_void_p(0x10002), 4, 1024, 1, GOOD, None) == -3
 
 
 def test_workspace_query_without_gpu_is_zero_or_positive(lib):
