@@ -289,6 +289,97 @@ int orc_accept_greedy(const float* logits, const int* tokens, const int* tree_pa
     return ORC_OK;
 }
 
+/* ------------------------------------------------------------------------------------------
+ * Stochastic (rejection-sampling) acceptance of a drafted chain.
+ * [abstract]: windowing preserves the target's verified output DISTRIBUTION; [verdict,
+ * referee_report.significance]: the losslessness is the standard speculative-decoding theorem.
+ * The pages do not restate the rule; this is the standard one (Leviathan, Kalman and Matias,
+ * "Fast Inference from Transformers via Speculative Decoding", ICML 2023, Algorithm 1; Chen et
+ * al., "Accelerating Large Language Model Decoding with Speculative Sampling", 2023):
+ *   for drafted token i = 1 .. n_q - 1 (x = tokens[i], proposed from the draft distribution
+ *   q_{i-1} = q[i - 1]; the target's distribution at that position is p_{i-1} = p[i - 1]):
+ *     accept x with probability min(1, p_{i-1}(x) / q_{i-1}(x));
+ *     on the first rejection emit a token drawn from norm(max(0, p_{i-1} - q_{i-1})) and stop;
+ *   when every draft is accepted, emit a token drawn from p_{n_q - 1} (the bonus).
+ * Randomness is an input and every decision is exact integer/fp64 arithmetic, so two
+ * implementations agree bit for bit:
+ *   acceptance: u = u_accept[i - 1] in [0, 2^24); accept iff u * q(x) < p(x) * 2^24, both
+ *     products exact in double (a 24-bit integer times a float32);
+ *   a draw from weights w(v) (w = max(0, p - q) computed in float32, or p): m(v) =
+ *     floor(w(v) * 2^40) as a 64-bit integer, M = sum_v m(v), t = floor(u_sample * M / 2^32)
+ *     with u_sample a 32-bit integer; emit the smallest v with m(0) + ... + m(v) > t.  If the
+ *     residual has M = 0 the draw uses p instead; if that is 0 too it emits token 0.
+ * Inputs: p [B, n_q, V] and q [B, n_q - 1, V] float32 probabilities (entries in [0, 1]);
+ * tokens [B, n_q] (tokens[0] = last committed token); u_accept [B, n_q - 1] (< 2^24);
+ * u_sample [B].  Outputs as orc_accept_greedy.
+ * ---------------------------------------------------------------------------------------- */
+#define ORC_FIX_SCALE 1099511627776.0   /* 2^40 */
+
+static uint64_t fix40(float w) {
+    if (!(w > 0.0f)) return 0;
+    return (uint64_t)((double)w * ORC_FIX_SCALE);     /* truncation = floor for w >= 0 */
+}
+
+/* The inverse-CDF draw described above over weights w; returns -1 when every m(v) is 0. */
+static int draw_fixed(const float* w, int V, uint32_t u_sample) {
+    uint64_t M = 0;
+    for (int v = 0; v < V; ++v) M += fix40(w[v]);
+    if (M == 0) return -1;
+    const unsigned __int128 prod = (unsigned __int128)u_sample * (unsigned __int128)M;
+    const uint64_t t = (uint64_t)(prod >> 32);
+    uint64_t c = 0;
+    for (int v = 0; v < V; ++v) {
+        c += fix40(w[v]);
+        if (c > t) return v;
+    }
+    return V - 1;   /* not reached: t < M */
+}
+
+int orc_accept_stochastic(const float* p, const float* q, const int* tokens,
+                          const uint32_t* u_accept, const uint32_t* u_sample,
+                          int B, int n_q, int V, int* accepted, int* n_accepted) {
+    if (B <= 0 || n_q <= 0 || V <= 0) return ORC_ERR_ARG;
+    float* w = (float*)malloc(sizeof(float) * (size_t)V);
+    if (!w) return ORC_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        const int* tok = tokens + (size_t)b * n_q;
+        int* acc = accepted + (size_t)b * n_q;
+        for (int i = 0; i < n_q; ++i) acc[i] = -1;
+        int n = 0, rejected_at = -1;
+        for (int i = 1; i < n_q; ++i) {
+            const int x = tok[i];
+            const float* pr = p + ((size_t)b * n_q + (i - 1)) * (size_t)V;
+            const float* qr = q + ((size_t)b * (n_q - 1) + (i - 1)) * (size_t)V;
+            const double px = (x >= 0 && x < V) ? (double)pr[x] : 0.0;
+            const double qx = (x >= 0 && x < V) ? (double)qr[x] : 0.0;
+            const double u = (double)u_accept[(size_t)b * (n_q - 1) + (i - 1)];
+            if (u * qx < px * 16777216.0) {
+                acc[n++] = x;
+            } else {
+                rejected_at = i;
+                break;
+            }
+        }
+        int y;
+        if (rejected_at > 0) {
+            const float* pr = p + ((size_t)b * n_q + (rejected_at - 1)) * (size_t)V;
+            const float* qr = q + ((size_t)b * (n_q - 1) + (rejected_at - 1)) * (size_t)V;
+            for (int v = 0; v < V; ++v) {
+                const float d = pr[v] - qr[v];
+                w[v] = d > 0.0f ? d : 0.0f;
+            }
+            y = draw_fixed(w, V, u_sample[b]);
+            if (y < 0) y = draw_fixed(pr, V, u_sample[b]);
+        } else {
+            y = draw_fixed(p + ((size_t)b * n_q + (n_q - 1)) * (size_t)V, V, u_sample[b]);
+        }
+        acc[n++] = y < 0 ? 0 : y;
+        n_accepted[b] = n;
+    }
+    free(w);
+    return ORC_OK;
+}
+
 /* Number of OpenMP threads the oracle would use (1 without OpenMP). */
 int orc_max_threads(void) {
 #ifdef _OPENMP

@@ -53,6 +53,8 @@ def _load():
         lib.orc_attention.restype = I
         lib.orc_accept_greedy.argtypes = [P, P, P, I, I, I, P, P]
         lib.orc_accept_greedy.restype = I
+        lib.orc_accept_stochastic.argtypes = [P, P, P, P, P, I, I, I, P, P]
+        lib.orc_accept_stochastic.restype = I
         lib.orc_max_threads.argtypes = []
         lib.orc_max_threads.restype = I
         _lib = lib
@@ -152,4 +154,25 @@ def accept_greedy(logits, tokens, tree_parent=None):
                                    _ptr(accepted), _ptr(n_acc))
     if rc != 0:
         raise ValueError("orc_accept_greedy: bad arguments")
+    return accepted, n_acc
+
+
+def accept_stochastic(p, q, tokens, u_accept, u_sample):
+    """Rejection-sampling acceptance of drafted chains.  p: f32 [B, n_q, V] target
+    probabilities; q: f32 [B, n_q - 1, V] draft probabilities; tokens: int32 [B, n_q];
+    u_accept: uint32 [B, n_q - 1] (< 2^24); u_sample: uint32 [B].  Returns (accepted int32
+    [B, n_q] padded with -1, n_accepted int32 [B])."""
+    p = _c(p, np.float32)
+    tokens = _c(tokens, np.int32)
+    B, n_q, V = p.shape
+    q = _c(q, np.float32).reshape(B, n_q - 1, V)
+    u_accept = _c(u_accept, np.uint32).reshape(B, n_q - 1)
+    u_sample = _c(u_sample, np.uint32).reshape(B)
+    assert tokens.shape == (B, n_q)
+    accepted = np.empty((B, n_q), dtype=np.int32)
+    n_acc = np.empty((B,), dtype=np.int32)
+    rc = _load().orc_accept_stochastic(_ptr(p), _ptr(q), _ptr(tokens), _ptr(u_accept), _ptr(u_sample),
+                                       B, n_q, V, _ptr(accepted), _ptr(n_acc))
+    if rc != 0:
+        raise ValueError("orc_accept_stochastic: bad arguments")
     return accepted, n_acc

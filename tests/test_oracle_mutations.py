@@ -14,6 +14,7 @@ from oracle.build_oracle import SRC
 import tests.test_oracle_accept as t_acc
 import tests.test_oracle_attention as t_att
 import tests.test_oracle_ring as t_ring
+import tests.test_oracle_stochastic as t_sto
 import tests.test_oracle_tree as t_tree
 import tests.test_oracle_window as t_win
 
@@ -35,6 +36,13 @@ MUTATIONS = [
     ("argmax_last_tie", "if (row[x] > bv)", "if (row[x] >= bv)"),
     ("tree_highest_child", "if (par[c] == cur && tok[c] == t[cur]) { next = c; break; }",
      "if (par[c] == cur && tok[c] == t[cur]) { next = c; }"),
+    ("stoch_residual_is_target", "const float d = pr[v] - qr[v];", "const float d = pr[v];"),
+    ("stoch_ratio_inverted", "if (u * qx < px * 16777216.0)", "if (u * px < qx * 16777216.0)"),
+    ("stoch_bonus_first_row", "y = draw_fixed(p + ((size_t)b * n_q + (n_q - 1)) * (size_t)V",
+     "y = draw_fixed(p + ((size_t)b * n_q + 0) * (size_t)V"),
+    ("stoch_rows_shifted", "const float* pr = p + ((size_t)b * n_q + (i - 1)) * (size_t)V;",
+     "const float* pr = p + ((size_t)b * n_q + i) * (size_t)V;"),
+    ("stoch_draw_off_by_one", "if (c > t) return v;", "if (c >= t) return v;"),
 ]
 
 PINS = [
@@ -55,6 +63,11 @@ PINS = [
     lambda: t_acc.test_chain_brute_force_all_drafts(2),
     lambda: t_acc.test_lossless_tree("random", 3),
     t_acc.test_tree_brute_force_small_vocab,
+    lambda: t_sto.test_emitted_token_is_distributed_as_the_target(0),
+    lambda: t_sto.test_emitted_token_is_distributed_as_the_target(3),
+    t_sto.test_second_position_uses_the_second_rows,
+    t_sto.test_disjoint_supports_reject_and_resample_from_the_target,
+    t_sto.test_acceptance_threshold_is_p_over_q,
 ]
 
 
