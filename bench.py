@@ -318,6 +318,26 @@ def run_gpu(args):
         "accept_greedy": kstat(lw.get("accept"), w.B * n_q_v * w.vocab * 4),
     }
 
+    # ---- stochastic acceptance on the step's verify nodes (softmax probabilities in) ----------
+    if not w.tree_nodes:
+        gs = torch.Generator(device=device)
+        gs.manual_seed(w.seed + 5)
+        p_ = torch.softmax(torch.randn((w.B, n_q_v, w.vocab), generator=gs, device=device), -1)
+        q_ = torch.softmax(torch.randn((w.B, n_q_v - 1, w.vocab), generator=gs, device=device), -1)
+        ua = torch.randint(0, 1 << 24, (w.B, n_q_v - 1), generator=gs, device=device, dtype=torch.int32)
+        us = torch.randint(-(1 << 31), (1 << 31) - 1, (w.B,), generator=gs, device=device, dtype=torch.int32)
+        acc_, nacc_ = api.accept_stochastic(p_, q_, step.b.tokens, ua, us)
+        ev = []
+        for _ in range(50):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            api.accept_stochastic(p_, q_, step.b.tokens, ua, us, accepted=acc_, n_accepted=nacc_)
+            e1.record()
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        assert api.device_status() == 0
+        kernels["accept_stochastic"] = kstat([a.elapsed_time(c) for a, c in ev[5:]], 2 * w.B * w.vocab * 4)
+
     # ---- windowed draft with a cold L2: rotate over ring copies larger than 2x L2 ----------
     cold = None
     if "ring_k" in shared:

@@ -171,6 +171,36 @@ WMTP_API int accept_greedy(const float* logits, const int32_t* tokens, const int
                   wmtp_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * accept_stochastic -- lossless acceptance of a drafted chain under sampling (rejection rule).
+ * [abstract]: the target's verified output distribution is preserved; [verdict,
+ * referee_report.significance]: the losslessness is the standard speculative-decoding theorem.
+ * The pages do not restate the rule; this is the standard one (Leviathan, Kalman and Matias,
+ * ICML 2023; Chen et al., 2023): draft i (x = tokens[b, i], proposed from q[b, i-1, :]) is kept
+ * with probability min(1, p[b, i-1, x] / q[b, i-1, x]); at the first rejection one token is drawn
+ * from norm(max(0, p[b, i-1, :] - q[b, i-1, :])); when all n_q - 1 drafts are kept, a bonus token
+ * is drawn from p[b, n_q-1, :].  The emitted tokens then follow the target's distributions.
+ *   Randomness is an input, and every decision is exact integer/double arithmetic (so results
+ *   are reproducible bit for bit):  keep iff u_accept[b, i-1] * q(x) < p(x) * 2^24, with
+ *   u_accept < 2^24;  a draw over weights w takes m(v) = floor(w(v) * 2^40) as 64-bit integers,
+ *   M = sum_v m(v), t = floor(u_sample[b] * M / 2^32), and emits the smallest v whose running sum
+ *   m(0) + ... + m(v) exceeds t (weights below 2^-40 are never drawn).  max(0, p - q) is computed
+ *   in float32.  A rejection with no residual mass (possible only when p and q do not sum to the
+ *   same total) draws from p instead; a row with no mass at all emits token 0.
+ *   p         [B, n_q, V] float   target probabilities (entries in [0, 1]) at the n_q positions
+ *   q         [B, n_q - 1, V] float   draft probabilities of the drafted positions (NULL if n_q = 1)
+ *   tokens    [B, n_q] int32      tokens[b, 0] = last committed token, then the drafts
+ *   u_accept  [B, n_q - 1] uint32 (NULL if n_q = 1);  u_sample [B] uint32
+ *   accepted  [B, n_q] int32 out (-1 padded);  n_accepted [B] int32 out (1 .. n_q)
+ *   A drafted token outside [0, V) is rejected and recorded as WMTP_ERR_DEVICE_INDEX in the
+ *   device status word.
+ *   Errors: WMTP_ERR_ARG (null pointers, B < 1, n_q < 1, n_q > 64, V < 1, V >= 2^24),
+ *           WMTP_ERR_ALIGN, WMTP_ERR_CUDA. */
+WMTP_API int accept_stochastic(const float* p, const float* q, const int32_t* tokens,
+                               const uint32_t* u_accept, const uint32_t* u_sample,
+                               int B, int n_q, int V, int32_t* accepted, int32_t* n_accepted,
+                               wmtp_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * draft_attn_window_noalloc -- draft_attn_window without a caller-supplied workspace.
  * The paper has no counterpart: this entry point exists for callers that cannot allocate device
  * memory on their decode path -- engines that plan every buffer at start-up and forbid later

@@ -45,6 +45,7 @@ _SIGNATURES = {
     "wmtp_device_status": ([P], I),
     "wmtp_launch_count": ([], ctypes.c_uint64),
     "draft_attn_window_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P], I),
+    "accept_stochastic": ([P, P, P, P, P, I, I, I, P, P, P], I),
     "ring_kv_append_at": ([P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
     "spec_commit": ([P, P, I, I, P, I64, P, P, P, P, I, P, I, P], I),
     "wmtp_synth_draft_tokens": ([P, P, I, I64, I, I, U64, U64, U32, P, P], I),

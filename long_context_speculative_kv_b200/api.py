@@ -241,3 +241,29 @@ def synth_target_logits(history, n_tokens, tokens, vocab: int, target_seed: int,
         _ptr(history), _ptr(n_tokens), B, history.shape[1], _ptr(tokens), _ptr(tree_parent), n_q,
         int(vocab), int(target_seed) & 0xFFFFFFFFFFFFFFFF, _ptr(logits), _stream(stream)))
     return logits
+
+
+def accept_stochastic(p, q, tokens, u_accept, u_sample, accepted=None, n_accepted=None, stream=None):
+    """Rejection-sampling acceptance of drafted chains (see wmtp.h).  p [B, n_q, V] and
+    q [B, n_q - 1, V] float32 probabilities; tokens [B, n_q] int32; u_accept [B, n_q - 1] and
+    u_sample [B] 32-bit integers (int32 or uint32 tensors holding the bit patterns)."""
+    _want(p, torch.float32, "p", 3)
+    _want(tokens, torch.int32, "tokens", 2)
+    B, n_q, V = p.shape
+    if n_q > 1:
+        _want(q, torch.float32, "q", 3)
+        if q.shape != (B, n_q - 1, V):
+            raise ValueError("accept_stochastic: q must be [B, n_q - 1, V]")
+        if u_accept.dtype not in (torch.int32, torch.uint32) or u_accept.shape != (B, n_q - 1) \
+                or not u_accept.is_contiguous() or not u_accept.is_cuda:
+            raise TypeError("u_accept: expected a contiguous [B, n_q - 1] 32-bit CUDA tensor")
+    if u_sample.dtype not in (torch.int32, torch.uint32) or u_sample.shape != (B,) or not u_sample.is_cuda:
+        raise TypeError("u_sample: expected a [B] 32-bit CUDA tensor")
+    if accepted is None:
+        accepted = torch.empty((B, n_q), dtype=torch.int32, device=p.device)
+    if n_accepted is None:
+        n_accepted = torch.empty((B,), dtype=torch.int32, device=p.device)
+    check("accept_stochastic", lib().accept_stochastic(
+        _ptr(p), _ptr(q) if n_q > 1 else None, _ptr(tokens), _ptr(u_accept) if n_q > 1 else None,
+        _ptr(u_sample), B, n_q, V, _ptr(accepted), _ptr(n_accepted), _stream(stream)))
+    return accepted, n_accepted

@@ -583,9 +583,9 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 // ---------------------------------------------------------------------------------------------
 // lse_merge_kernel: combines the split partials of units that span several CTAs, and writes
 // empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block), 128
-// threads (one per head dim).  Partial s has weight 2^(lse_s - max_s lse_s); empty partials have
-// lse = -inf and weight 0.  The partials' LSEs are read by all threads in parallel, then every
-// thread sums its head dim over the partials with independent loads.
+// threads.  Partial s has weight 2^(lse_s - max_s lse_s); empty partials have lse = -inf and
+// weight 0.  The partials' LSEs are read by all threads in parallel; then each warp sums a
+// quarter of the partials with 16-byte loads and the four warp sums are combined per head dim.
 constexpr int kMaxParts = 1024;
 
 template <int SRC>
@@ -646,25 +646,50 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     for (int k = 1; k < kD / 32; ++k) mx = fmaxf(mx, s_red[k]);
     for (int k = d; k < np; k += kD) s_w[k] = (mx == -INFINITY) ? 0.f : exp2f(s_w[k] - mx);
     __syncthreads();
-    const float* o_base = a.ws_o + ((size_t)(c_lo + u) * a.rows_blk + rr) * kD + d;
-    const size_t kSlotStride = (size_t)a.rows_blk * kD;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, wsum = 0.f;
-    int k = 0;
-    for (; k + 4 <= np; k += 4) {
-        acc0 += s_w[k] * o_base[(size_t)k * kSlotStride];
-        acc1 += s_w[k + 1] * o_base[(size_t)(k + 1) * kSlotStride];
-        acc2 += s_w[k + 2] * o_base[(size_t)(k + 2) * kSlotStride];
-        acc3 += s_w[k + 3] * o_base[(size_t)(k + 3) * kSlotStride];
-        wsum += (s_w[k] + s_w[k + 1]) + (s_w[k + 2] + s_w[k + 3]);
+    // Each warp takes every 4th partial; lane l owns head dims [4l, 4l + 4) (one 16-byte load
+    // per partial, 512 contiguous bytes per warp), four partials in flight per step.
+    const int warp = d >> 5, lane = d & 31;
+    const float4* o_base = reinterpret_cast<const float4*>(
+        a.ws_o + ((size_t)(c_lo + u) * a.rows_blk + rr) * kD) + lane;
+    const size_t kSlotStride4 = (size_t)a.rows_blk * (kD / 4);
+    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+    float wsum = 0.f;
+    int k = warp;
+    for (; k + 12 < np; k += 16) {
+        const float4 x0 = o_base[(size_t)k * kSlotStride4];
+        const float4 x1 = o_base[(size_t)(k + 4) * kSlotStride4];
+        const float4 x2 = o_base[(size_t)(k + 8) * kSlotStride4];
+        const float4 x3 = o_base[(size_t)(k + 12) * kSlotStride4];
+        const float w0 = s_w[k], w1 = s_w[k + 4], w2 = s_w[k + 8], w3 = s_w[k + 12];
+        acc0.x += w0 * x0.x + w2 * x2.x; acc0.y += w0 * x0.y + w2 * x2.y;
+        acc0.z += w0 * x0.z + w2 * x2.z; acc0.w += w0 * x0.w + w2 * x2.w;
+        acc1.x += w1 * x1.x + w3 * x3.x; acc1.y += w1 * x1.y + w3 * x3.y;
+        acc1.z += w1 * x1.z + w3 * x3.z; acc1.w += w1 * x1.w + w3 * x3.w;
+        wsum += (w0 + w1) + (w2 + w3);
     }
-    for (; k < np; ++k) {
-        acc0 += s_w[k] * o_base[(size_t)k * kSlotStride];
-        wsum += s_w[k];
+    for (; k < np; k += 4) {
+        const float4 x0 = o_base[(size_t)k * kSlotStride4];
+        const float w0 = s_w[k];
+        acc0.x += w0 * x0.x; acc0.y += w0 * x0.y; acc0.z += w0 * x0.z; acc0.w += w0 * x0.w;
+        wsum += w0;
     }
-    const float acc = (acc0 + acc1) + (acc2 + acc3);
-    const float res = wsum > 0.f ? acc / wsum : 0.f;
+    __shared__ float4 s_acc[kD / 32][32];
+    __shared__ float s_wsum[kD / 32];
+    s_acc[warp][lane] = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+    if (lane == 0) s_wsum[warp] = wsum;
+    __syncthreads();
+    // thread d sums head dim d over the four warps
+    const float* s_flat = reinterpret_cast<const float*>(s_acc);
+    const int l4 = d >> 2, c4 = d & 3;
+    float acc = 0.f, wt = 0.f;
+#pragma unroll
+    for (int g = 0; g < kD / 32; ++g) {
+        acc += s_flat[(g * 32 + l4) * 4 + c4];
+        wt += s_wsum[g];
+    }
+    const float res = wt > 0.f ? acc / wt : 0.f;
     a.out[orow * kD + d] = __float2bfloat16_rn(res);
-    if (a.lse != nullptr && d == 0) a.lse[orow] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
+    if (a.lse != nullptr && d == 0) a.lse[orow] = wt > 0.f ? (mx + log2f(wt)) * kLn2 : -INFINITY;
 }
 
 }  // namespace wmtp

@@ -541,6 +541,28 @@ int accept_greedy(const float* logits, const int32_t* tokens, const int32_t* tre
                   logits, tokens, tree_parent, n_q, V, accepted, n_accepted);
 }
 
+int accept_stochastic(const float* p, const float* q, const int32_t* tokens, const uint32_t* u_accept,
+                      const uint32_t* u_sample, int B, int n_q, int V, int32_t* accepted,
+                      int32_t* n_accepted, wmtp_stream_t stream) {
+    if (p == nullptr || tokens == nullptr || u_sample == nullptr || accepted == nullptr ||
+        n_accepted == nullptr)
+        return WMTP_ERR_ARG;
+    if (B < 1 || n_q < 1 || n_q > WMTP_MAX_QUERIES || V < 1 || V >= (1 << 24)) return WMTP_ERR_ARG;
+    if (n_q > 1 && (q == nullptr || u_accept == nullptr)) return WMTP_ERR_ARG;
+    if (!aligned(p, 4) || !aligned(tokens, 4) || !aligned(u_sample, 4) || !aligned(accepted, 4) ||
+        !aligned(n_accepted, 4) || (q && !aligned(q, 4)) || (u_accept && !aligned(u_accept, 4)))
+        return WMTP_ERR_ALIGN;
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (V <= 4096)
+        return launch(accept_stochastic_kernel<256>, dim3(B), dim3(256), 0, st, p, q, tokens,
+                      u_accept, u_sample, n_q, V, accepted, n_accepted);
+    return launch(accept_stochastic_kernel<1024>, dim3(B), dim3(1024), 0, st, p, q, tokens, u_accept,
+                  u_sample, n_q, V, accepted, n_accepted);
+}
+
 int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,
                               const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D,
                               int n_sink, int window, int capacity, float sm_scale, wmtp_bf16* out,

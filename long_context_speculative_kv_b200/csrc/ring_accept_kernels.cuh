@@ -122,3 +122,130 @@ accept_greedy_kernel(const float* __restrict__ logits, const int* __restrict__ t
 }
 
 }  // namespace wmtp
+
+namespace wmtp {
+
+// ---------------------------------------------------------------------------------------------
+// Stochastic acceptance (AI field-notes abstract for 2607.21535: the target's verified output
+// distribution is preserved; Pith verdict, referee_report.significance: the standard
+// speculative-decoding theorem).  The standard rejection rule (Leviathan, Kalman and Matias,
+// ICML 2023; Chen et al., 2023): draft i is kept with probability min(1, p_{i-1}(x) / q_{i-1}(x));
+// at the first rejection a token is drawn from norm(max(0, p_{i-1} - q_{i-1})); after all gamma
+// drafts a bonus token is drawn from p_gamma.  Randomness comes in as integers and every
+// decision is exact: keep iff u * q(x) < p(x) * 2^24 (u < 2^24; both products exact in double);
+// a draw over weights w uses m(v) = floor(w(v) * 2^40) (64-bit integers), M = sum m,
+// t = floor(u_sample * M / 2^32) and picks the smallest v whose running sum of m exceeds t.
+// With no residual mass (M = 0) the draw uses p; with none there either it emits token 0.
+// One CTA per request: thread 0 walks the drafts; the draw is a block-wide integer scan
+// (each thread owns a contiguous chunk of the vocabulary), so the result does not depend on
+// the summation order.
+__device__ __forceinline__ unsigned long long fix40(float w) {
+    if (!(w > 0.f)) return 0ull;
+    return (unsigned long long)((double)w * 1099511627776.0);      // 2^40, truncating
+}
+
+// w(v) = max(0, a[v] - b[v]) when b != nullptr, else a[v].
+__device__ __forceinline__ float draw_weight(const float* a, const float* b, int v) {
+    if (b == nullptr) return a[v];
+    const float d = __fsub_rn(a[v], b[v]);
+    return d > 0.f ? d : 0.f;
+}
+
+template <int NT>
+__device__ int block_draw(const float* a, const float* b, int V, unsigned int u_sample,
+                          unsigned long long* s_warp, int* s_y) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chunk = (V + NT - 1) / NT;
+    const int v0 = tid * chunk;
+    const int v1 = min(V, v0 + chunk);
+    unsigned long long local = 0;
+    for (int v = v0; v < v1; ++v) local += fix40(draw_weight(a, b, v));
+    // block-wide exclusive scan of the per-thread sums (integers: exact in any order)
+    unsigned long long incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    if (tid == 0) *s_y = -1;
+    __syncthreads();
+    unsigned long long base = 0, M = 0;
+    for (int w = 0; w < NT / 32; ++w) {
+        if (w < warp) base += s_warp[w];
+        M += s_warp[w];
+    }
+    const unsigned long long excl = base + incl - local;
+    if (M != 0) {
+        const unsigned long long t =
+            (unsigned long long)u_sample * (M >> 32) + (((unsigned long long)u_sample * (M & 0xffffffffull)) >> 32);
+        if (excl <= t && t < excl + local) {
+            unsigned long long c = excl;
+            for (int v = v0; v < v1; ++v) {
+                c += fix40(draw_weight(a, b, v));
+                if (c > t) { *s_y = v; break; }
+            }
+        }
+    }
+    __syncthreads();
+    const int y = *s_y;
+    __syncthreads();                       // s_warp / s_y may be reused by the next draw
+    return y;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT)
+accept_stochastic_kernel(const float* __restrict__ p, const float* __restrict__ q,
+                         const int* __restrict__ tokens, const unsigned int* __restrict__ u_accept,
+                         const unsigned int* __restrict__ u_sample, int n_q, int V,
+                         int* __restrict__ accepted, int* __restrict__ n_accepted) {
+    __shared__ unsigned long long s_warp[NT / 32];
+    __shared__ int s_y, s_rej, s_n;
+    pdl_launch_dependents();
+    pdl_wait();
+    const int b = blockIdx.x;
+    const int* tok = tokens + (size_t)b * n_q;
+    if (threadIdx.x == 0) {
+        int n = 0, rej = -1;
+        for (int i = 1; i < n_q; ++i) {
+            const int x = tok[i];
+            double px = 0.0, qx = 0.0;
+            if (x >= 0 && x < V) {
+                px = (double)p[((size_t)b * n_q + (i - 1)) * (size_t)V + x];
+                qx = (double)q[((size_t)b * (n_q - 1) + (i - 1)) * (size_t)V + x];
+            } else {
+                flag_status(kStatusDeviceIndex);
+            }
+            const double u = (double)u_accept[(size_t)b * (n_q - 1) + (i - 1)];
+            if (u * qx < px * 16777216.0) {
+                ++n;
+            } else {
+                rej = i;
+                break;
+            }
+        }
+        s_n = n;
+        s_rej = rej;
+    }
+    __syncthreads();
+    const int n = s_n, rej = s_rej;
+    int y;
+    if (rej > 0) {
+        const float* pr = p + ((size_t)b * n_q + (rej - 1)) * (size_t)V;
+        const float* qr = q + ((size_t)b * (n_q - 1) + (rej - 1)) * (size_t)V;
+        y = block_draw<NT>(pr, qr, V, u_sample[b], s_warp, &s_y);
+        if (y < 0) y = block_draw<NT>(pr, nullptr, V, u_sample[b], s_warp, &s_y);
+    } else {
+        y = block_draw<NT>(p + ((size_t)b * n_q + (n_q - 1)) * (size_t)V, nullptr, V, u_sample[b],
+                           s_warp, &s_y);
+    }
+    if (threadIdx.x == 0) {
+        int* acc = accepted + (size_t)b * n_q;
+        for (int j = 0; j < n; ++j) acc[j] = tok[j + 1];
+        acc[n] = y < 0 ? 0 : y;
+        for (int j = n + 1; j < n_q; ++j) acc[j] = -1;
+        n_accepted[b] = n + 1;
+    }
+}
+
+}  // namespace wmtp

@@ -29,7 +29,7 @@ def test_header_declares_the_five_calls_and_helpers():
     assert {"ring_kv_append", "draft_attn_window", "draft_attn_full", "verify_attn",
             "accept_greedy", "wmtp_workspace_bytes", "wmtp_status_string",
             "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc",
-            "ring_kv_append_at", "spec_commit", "wmtp_synth_draft_tokens",
+            "accept_stochastic", "ring_kv_append_at", "spec_commit", "wmtp_synth_draft_tokens",
             "wmtp_synth_target_logits"} == names
     assert set(_lib._SIGNATURES) == names
 
@@ -99,6 +99,16 @@ def test_accept_host_checks(lib):
     assert a(GOOD, GOOD, None, 1, 65, 1024, GOOD, GOOD, None) == -1
     assert a(GOOD, GOOD, None, 1, 4, 0, GOOD, GOOD, None) == -1
     assert a(ctypes.c_void_p(0x10002), GOOD, None, 1, 4, 1024, GOOD, GOOD, None) == -3
+
+
+def test_stochastic_accept_host_checks(lib):
+    a = lib.accept_stochastic
+    # (p, q, tokens, u_acc, u_samp, B, n_q, V, accepted, n_accepted, stream)
+    assert a(GOOD, None, GOOD, None, GOOD, 1, 4, 1024, GOOD, GOOD, None) == -1       # q missing
+    assert a(GOOD, GOOD, GOOD, GOOD, GOOD, 1, 65, 1024, GOOD, GOOD, None) == -1      # n_q > 64
+    assert a(GOOD, GOOD, GOOD, GOOD, GOOD, 1, 4, 1 << 24, GOOD, GOOD, None) == -1    # V >= 2^24
+    assert a(GOOD, GOOD, GOOD, GOOD, None, 1, 4, 1024, GOOD, GOOD, None) == -1       # u_sample
+    assert a(GOOD, GOOD, ctypes.c_void_p(0x10002), GOOD, GOOD, 1, 4, 1024, GOOD, GOOD, None) == -3
 
 
 def test_loop_host_checks(lib):
