@@ -55,6 +55,10 @@ def _load():
         lib.orc_accept_greedy.restype = I
         lib.orc_accept_stochastic.argtypes = [P, P, P, P, P, I, I, I, P, P]
         lib.orc_accept_stochastic.restype = I
+        lib.orc_e4m3_value.argtypes = [ctypes.c_uint]
+        lib.orc_e4m3_value.restype = ctypes.c_double
+        lib.orc_e4m3_decode.argtypes = [P, ctypes.c_size_t, P]
+        lib.orc_e4m3_decode.restype = None
         lib.orc_max_threads.argtypes = []
         lib.orc_max_threads.restype = I
         _lib = lib
@@ -176,3 +180,38 @@ def accept_stochastic(p, q, tokens, u_accept, u_sample):
     if rc != 0:
         raise ValueError("orc_accept_stochastic: bad arguments")
     return accepted, n_acc
+
+
+def e4m3_value(code: int) -> float:
+    """The value of one OCP E4M3 code (NaN for S.1111.111)."""
+    return float(_load().orc_e4m3_value(int(code) & 0xFF))
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of an array of E4M3 codes (uint8), same shape."""
+    codes = _c(codes, np.uint8)
+    out = np.empty(codes.shape, dtype=np.float64)
+    _load().orc_e4m3_decode(_ptr(codes), codes.size, _ptr(out))
+    return out
+
+
+def _f64_to_bf16_bits_exact(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of float64 values that bf16 represents exactly (every finite E4M3
+    value does: 3 mantissa bits, exponents -9 .. 8); NaN stays NaN."""
+    f = x.astype(np.float32)
+    bits = f.view(np.uint32)
+    assert not np.any((bits & 0xFFFF)[np.isfinite(f)]), "value not exactly representable in bf16"
+    return (bits >> 16).astype(np.uint16)
+
+
+def attention_kv8(q, k8, v8, kv_len, mode: int, sm_scale: float, k_scale: float, v_scale: float,
+                  n_sink: int = 0, window: int = 0, tree_parent=None, rows=None, n_threads: int = 0):
+    """attention() over fp8 (E4M3) keys and values: key = k_scale * e4m3(k8), value =
+    v_scale * e4m3(v8).  k8, v8: uint8 [B, Hkv, Lmax, D] in logical order.  The decoded codes are
+    exact bf16 values, the key scale multiplies every score (folded into sm_scale) and the value
+    scale every output, so this is the fp64 definition on the dequantised cache."""
+    kb = _f64_to_bf16_bits_exact(e4m3_decode(k8))
+    vb = _f64_to_bf16_bits_exact(e4m3_decode(v8))
+    out, lse = attention(q, kb, vb, kv_len, mode, float(sm_scale) * float(k_scale), n_sink=n_sink,
+                         window=window, tree_parent=tree_parent, rows=rows, n_threads=n_threads)
+    return out * float(v_scale), lse

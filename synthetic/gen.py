@@ -201,3 +201,33 @@ def hash_draft_tokens(target_seed: int, draft_seed: int, prefix: Sequence[int], 
         r = int(splitmix64(z)) % (vocab - 1)
         out.append(greedy if agree else (greedy + 1 + r) % vocab)
     return out
+
+
+# ----------------------------------------------------------------------------- fp8 (E4M3) codes
+def _e4m3_grid() -> np.ndarray:
+    """Values of the positive E4M3 codes 0 .. 126 (OCP OFP8: bias 7, subnormals (m/8) 2^-6,
+    S.1111.111 reserved for NaN)."""
+    vals = [m / 8.0 * 2.0 ** -6 for m in range(8)]
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                break
+            vals.append((1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.asarray(vals, dtype=np.float64)
+
+
+_E4M3_GRID = _e4m3_grid()
+
+
+def e4m3_codes(x) -> np.ndarray:
+    """uint8 E4M3 codes of x: round to nearest, ties to the even code, saturating at +-448
+    (how an fp8 KV cache writer quantises); NaN -> 0x7F."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    idx = np.clip(np.searchsorted(_E4M3_GRID, a), 1, len(_E4M3_GRID) - 1)
+    lo, hi = _E4M3_GRID[idx - 1], _E4M3_GRID[idx]
+    dlo, dhi = a - lo, hi - a
+    take_hi = (dhi < dlo) | ((dhi == dlo) & (idx % 2 == 0))
+    code = np.where(take_hi, idx, idx - 1).astype(np.uint8)
+    code = np.where(x < 0, code | np.uint8(0x80), code).astype(np.uint8)
+    return np.where(np.isnan(x), np.uint8(0x7F), code).astype(np.uint8)

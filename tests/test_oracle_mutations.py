@@ -13,6 +13,7 @@ from oracle.build_oracle import SRC
 
 import tests.test_oracle_accept as t_acc
 import tests.test_oracle_attention as t_att
+import tests.test_oracle_fp8 as t_fp8
 import tests.test_oracle_ring as t_ring
 import tests.test_oracle_stochastic as t_sto
 import tests.test_oracle_tree as t_tree
@@ -43,6 +44,11 @@ MUTATIONS = [
     ("stoch_rows_shifted", "const float* pr = p + ((size_t)b * n_q + (i - 1)) * (size_t)V;",
      "const float* pr = p + ((size_t)b * n_q + i) * (size_t)V;"),
     ("stoch_draw_off_by_one", "if (c > t) return v;", "if (c >= t) return v;"),
+    ("e4m3_bias_8", "else mag = ldexp(1.0 + (double)m / 8.0, (int)e - 7);",
+     "else mag = ldexp(1.0 + (double)m / 8.0, (int)e - 8);"),
+    ("e4m3_subnormal_scale", "if (e == 0u) mag = ldexp((double)m / 8.0, -6);",
+     "if (e == 0u) mag = ldexp((double)m / 8.0, -7);"),
+    ("e4m3_no_nan", "if (e == 15u && m == 7u) return NAN;", "if (e == 16u && m == 7u) return NAN;"),
 ]
 
 PINS = [
@@ -68,6 +74,8 @@ PINS = [
     t_sto.test_second_position_uses_the_second_rows,
     t_sto.test_disjoint_supports_reject_and_resample_from_the_target,
     t_sto.test_acceptance_threshold_is_p_over_q,
+    t_fp8.test_published_e4m3_values,
+    t_fp8.test_e4m3_codes_are_ordered_and_finite_except_nan,
 ]
 
 
