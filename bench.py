@@ -42,6 +42,7 @@ def parse():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-loop", action="store_true", help="skip the decode-loop measurement")
+    p.add_argument("--no-fp8", action="store_true", help="skip the fp8-KV measurement")
     p.add_argument("--agree", type=float, default=0.8,
                    help="decode loop: probability a synthetic draft proposal is the target's token")
     p.add_argument("--context", type=int, default=0, help="override the committed context (profiling cases)")
@@ -521,6 +522,48 @@ def run_gpu(args):
             100 * (loop_res["native"]["us_per_step"] / loop_res["windowed"]["us_per_step"] - 1), 2)
         loop_res["per_token_speedup"] = round(loop_res["native"]["us_per_token"] / loop_res["windowed"]["us_per_token"], 4)
 
+    # ---- fp8 (E4M3) KV: the same step with every K/V cache in fp8 ---------------------------
+    fp8_res = None
+    if not args.no_fp8:
+        shared8 = workload.shared_inputs(w, device, max_nq_verify=n_q_v, max_gamma=args.gamma,
+                                         window=window, n_layers=args.layers or None, kv8=True)
+        st8 = DecodeStep(StepBuffers(**workload.step_inputs(w, shared8, args.gamma, device)), args.gamma)
+        step, keep = st8, step
+        K8 = max(10, args.steps // 4)
+        for _ in range(2):
+            step.run("windowed")
+            step.run("native")
+        _, lg8w, _ = timed("windowed", K8)
+        _, lg8n, _ = timed("native", K8)
+        if use_graph:
+            gw8, _ = capture("windowed")
+            gn8, _ = capture("native")
+            m8w, m8n = timed_graph(gw8, K8), timed_graph(gn8, K8)
+            del gw8, gn8
+        else:
+            m8w, _, _ = timed("windowed", K8, with_log=False)
+            m8n, _, _ = timed("native", K8, with_log=False)
+        assert api.device_status() == 0
+        step = keep
+        l8w, l8n = per_label(lg8w), per_label(lg8n)
+        row8 = w.Hkv * w.D * 2                                 # K + V bytes of one position
+        fp8_res = {
+            "k_scale": st8.b.k_scale, "v_scale": st8.b.v_scale,
+            "windowed_us": round(max_ranks(m8w) * 1e3 / K8, 2),
+            "native_us": round(max_ranks(m8n) * 1e3 / K8, 2),
+            "kernels": {
+                "verify_attn_fp8": kstat(l8w.get("verify"), sum(L + n_q_v for L in lens) * row8),
+                "draft_attn_full_fp8_fwd": kstat(l8n.get("full_fwd"), sum(L + args.gamma + 2 for L in lens) * row8),
+                "draft_attn_window_fp8_fwd_inloop": kstat(
+                    l8w.get("window_fwd"),
+                    sum(acc.window_keys(L + args.gamma + 1, w.n_sink, window) for L in lens) * row8),
+            },
+        }
+        fp8_res["step_cost_reduction_pct"] = round(100 * (fp8_res["native_us"] / fp8_res["windowed_us"] - 1), 2)
+        fp8_res["windowed_speedup_over_bf16"] = round(us_w_local / fp8_res["windowed_us"], 4)
+        del st8, shared8
+        torch.cuda.empty_cache()
+
     # ---- KV accounting -------------------------------------------------------------------
     sb_w = acc.step_bytes(int(statistics.mean(lens)), args.gamma, n_q_v, w.Hkv, w.D, n_layers,
                           w.n_sink, window, windowed=True)
@@ -572,7 +615,7 @@ def run_gpu(args):
         "step_cost_ratio_native_over_windowed": round(ms_n_max / ms_w_max, 4),
         "step_cost_reduction_pct": round(100 * (ms_n_max / ms_w_max - 1), 2),
         "kernels": dict(kernels, draft_attn_window_fwd_cold=cold),
-        "gamma_sweep": sweep, "context_sweep": ctx_sweep, "decode_loop": loop_res,
+        "gamma_sweep": sweep, "context_sweep": ctx_sweep, "decode_loop": loop_res, "fp8_kv": fp8_res,
         "kv_accounting": accounting,
         "roofline": roofline, "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 3), "unit": "us/step",

@@ -201,6 +201,44 @@ WMTP_API int accept_stochastic(const float* p, const float* q, const int32_t* to
                                wmtp_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * fp8 (E4M3) KV variants.  [verdict, pith_extraction.forward_implications[4]]: windowing
+ * composes with KV quantisation (fp8), which halves the bytes every attention call streams.
+ *   K and V hold OCP E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ *   infinities), one byte per element, in the layouts of the bf16 calls:
+ *       ring K/V [B, Hkv, capacity, 128] uint8;  pools [num_pages, Hkv, 64, 128] uint8.
+ *   A key is k_scale times its code's value, a value v_scale times its code's value (one
+ *   scale per tensor, > 0).  q, out, lse, the workspace and every other argument are those of
+ *   the bf16 call of the same name; the workspace size is the same.  The kernels widen codes
+ *   and queries to fp16 exactly and accumulate in fp32, so results match attention over the
+ *   dequantised cache to the tolerance of the bf16 calls.  Codes of NaN (S.1111.111) must not
+ *   occur in keys or values that a query can see.
+ *   Errors: those of the bf16 call, plus WMTP_ERR_ARG for a scale <= 0 or not finite.
+ * ring_kv_append_fp8: ring_kv_append on fp8 rows (128 bytes per row and head). */
+WMTP_API int ring_kv_append_fp8(uint8_t* ring_k, uint8_t* ring_v, int64_t* ring_len,
+                                const uint8_t* k_new, const uint8_t* v_new,
+                                int B, int n_new, int Hkv, int D, int n_sink, int capacity,
+                                wmtp_stream_t stream);
+WMTP_API int draft_attn_window_fp8(const wmtp_bf16* q, const uint8_t* ring_k, const uint8_t* ring_v,
+                                   const int64_t* ring_len,
+                                   int B, int n_q, int Hq, int Hkv, int D, int n_sink, int window,
+                                   int capacity, float sm_scale, float k_scale, float v_scale,
+                                   wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                                   wmtp_stream_t stream);
+WMTP_API int draft_attn_full_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const uint8_t* v_pool,
+                                 const int32_t* page_table, const int32_t* kv_len,
+                                 int B, int n_q, int Hq, int Hkv, int D, int page_size, int max_pages,
+                                 int num_pages, float sm_scale, float k_scale, float v_scale,
+                                 wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                                 wmtp_stream_t stream);
+WMTP_API int verify_attn_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const uint8_t* v_pool,
+                             const int32_t* page_table, const int32_t* kv_len,
+                             const int32_t* tree_parent,
+                             int B, int n_q, int Hq, int Hkv, int D, int page_size, int max_pages,
+                             int num_pages, float sm_scale, float k_scale, float v_scale,
+                             wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                             wmtp_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * draft_attn_window_noalloc -- draft_attn_window without a caller-supplied workspace.
  * The paper has no counterpart: this entry point exists for callers that cannot allocate device
  * memory on their decode path -- engines that plan every buffer at start-up and forbid later

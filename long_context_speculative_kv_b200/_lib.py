@@ -46,6 +46,10 @@ _SIGNATURES = {
     "wmtp_launch_count": ([], ctypes.c_uint64),
     "draft_attn_window_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P], I),
     "accept_stochastic": ([P, P, P, P, P, I, I, I, P, P, P], I),
+    "ring_kv_append_fp8": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
+    "draft_attn_window_fp8": ([P, P, P, P, I, I, I, I, I, I, I, I, F, F, F, P, P, P, SZ, P], I),
+    "draft_attn_full_fp8": ([P, P, P, P, P, I, I, I, I, I, I, I, I, F, F, F, P, P, P, SZ, P], I),
+    "verify_attn_fp8": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, F, F, P, P, P, SZ, P], I),
     "ring_kv_append_at": ([P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
     "spec_commit": ([P, P, I, I, P, I64, P, P, P, P, I, P, I, P], I),
     "wmtp_synth_draft_tokens": ([P, P, I, I64, I, I, U64, U64, U32, P, P], I),

@@ -267,3 +267,87 @@ def accept_stochastic(p, q, tokens, u_accept, u_sample, accepted=None, n_accepte
         _ptr(p), _ptr(q) if n_q > 1 else None, _ptr(tokens), _ptr(u_accept) if n_q > 1 else None,
         _ptr(u_sample), B, n_q, V, _ptr(accepted), _ptr(n_accepted), _stream(stream)))
     return accepted, n_accepted
+
+
+# ----------------------------------------------------------------------------- fp8 (E4M3) KV
+_FP8_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _want8(t, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or t.dtype not in _FP8_DTYPES or t.dim() != ndim:
+        raise TypeError(f"{name}: expected a {ndim}-d uint8 / float8_e4m3fn tensor of E4M3 codes")
+    if not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous CUDA tensor")
+
+
+def ring_kv_append_fp8(ring_k, ring_v, ring_len, k_new, v_new, n_sink: int, stream=None) -> None:
+    """ring_kv_append on E4M3 rows: ring [B, Hkv, C, 128], new rows [B, n_new, Hkv, 128]."""
+    _want8(ring_k, "ring_k", 4)
+    _want8(ring_v, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    _want8(k_new, "k_new", 4)
+    _want8(v_new, "v_new", 4)
+    B, Hkv, C, D = ring_k.shape
+    n_new = k_new.shape[1]
+    if k_new.shape != (B, n_new, Hkv, D) or v_new.shape != k_new.shape or ring_v.shape != ring_k.shape:
+        raise ValueError("ring_kv_append_fp8: inconsistent shapes")
+    check("ring_kv_append_fp8", lib().ring_kv_append_fp8(
+        _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), _ptr(k_new), _ptr(v_new),
+        B, n_new, Hkv, D, int(n_sink), C, _stream(stream)))
+
+
+def draft_attn_window_fp8(q, ring_k, ring_v, ring_len, n_sink: int, window: int, sm_scale: float,
+                          k_scale: float, v_scale: float, ws: torch.Tensor, out=None, lse=None,
+                          want_lse: bool = True, stream=None):
+    _want(q, torch.bfloat16, "q", 4)
+    _want8(ring_k, "ring_k", 4)
+    _want8(ring_v, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    B, n_q, Hq, D = q.shape
+    _, Hkv, C, _ = ring_k.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_window_fp8", lib().draft_attn_window_fp8(
+        _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), B, n_q, Hq, Hkv, D, int(n_sink),
+        int(window), C, float(sm_scale), float(k_scale), float(v_scale), _ptr(out), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def _paged8_checks(q, k_pool, v_pool, page_table, kv_len):
+    _want(q, torch.bfloat16, "q", 4)
+    _want8(k_pool, "k_pool", 4)
+    _want8(v_pool, "v_pool", 4)
+    _want(page_table, torch.int32, "page_table", 2)
+    _want(kv_len, torch.int32, "kv_len", 1)
+    if v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool and v_pool differ in shape")
+
+
+def draft_attn_full_fp8(q, k_pool, v_pool, page_table, kv_len, sm_scale: float, k_scale: float,
+                        v_scale: float, ws: torch.Tensor, out=None, lse=None, want_lse: bool = True,
+                        stream=None):
+    _paged8_checks(q, k_pool, v_pool, page_table, kv_len)
+    B, n_q, Hq, D = q.shape
+    num_pages, Hkv, P, _ = k_pool.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_full_fp8", lib().draft_attn_full_fp8(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(kv_len), B, n_q, Hq, Hkv, D, P,
+        page_table.shape[1], num_pages, float(sm_scale), float(k_scale), float(v_scale), _ptr(out),
+        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def verify_attn_fp8(q, k_pool, v_pool, page_table, kv_len, sm_scale: float, k_scale: float,
+                    v_scale: float, ws: torch.Tensor, tree_parent=None, out=None, lse=None,
+                    want_lse: bool = True, stream=None):
+    _paged8_checks(q, k_pool, v_pool, page_table, kv_len)
+    if tree_parent is not None:
+        _want(tree_parent, torch.int32, "tree_parent", 2)
+    B, n_q, Hq, D = q.shape
+    num_pages, Hkv, P, _ = k_pool.shape
+    out, lse = _outs(q, out, lse, want_lse)
+    check("verify_attn_fp8", lib().verify_attn_fp8(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(kv_len), _ptr(tree_parent),
+        B, n_q, Hq, Hkv, D, P, page_table.shape[1], num_pages, float(sm_scale), float(k_scale),
+        float(v_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse

@@ -32,6 +32,8 @@ constexpr int kRowsPerBlock = 64;
 constexpr int kHalfBytes = kTileKeys * 64 * 2;      // one 64x64 bf16 box: 8 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;          // K or V tile: 16 KiB
 constexpr int kStageBytes = 2 * kTileBytes;         // K + V: 32 KiB
+constexpr int kTileBytes8 = kTileKeys * kD;         // fp8 K or V tile: one 128x64 byte box, 8 KiB
+constexpr int kStageBytes8 = 2 * kTileBytes8;       // fp8 K + V: 16 KiB
 constexpr int kMaxBatch = 256;
 constexpr float kLn2 = 0.693147180559945309f;
 
@@ -46,7 +48,8 @@ struct AttnArgs {
     int B, n_q, Hq, Hkv, G, n_rb;
     int rows_total;              // n_q * G
     int rows_blk;                // rows per unit (min(64, rows_total)): the workspace slot height
-    float scale_log2;            // sm_scale * log2(e)
+    float scale_log2;            // sm_scale * log2(e) (fp8 KV: times the key scale)
+    float v_scale;               // output multiplier (fp8 KV: the value scale; else 1)
     const int* tree_parent;      // [B, n_q] or null (chain / causal)
     // paged source
     const int* page_table;       // [B, max_pages]
@@ -211,9 +214,9 @@ __device__ __forceinline__ unsigned long long step_visibility(const AttnArgs& a,
 
 // ---------------------------------------------------------------------------------------------
 // Shared-memory layout (dynamic; stage buffers 1024-byte aligned for the 128-byte swizzle).
-template <int NMT, int NKG, int NSTAGE>
+template <int NMT, int NKG, int NSTAGE, bool KV8 = false>
 struct SmemLayout {
-    static constexpr int kStagesBytes = NSTAGE * kStageBytes;
+    static constexpr int kStagesBytes = NSTAGE * (KV8 ? kStageBytes8 : kStageBytes);
     static constexpr int kMergeStride = kD + 4;                      // floats per merge row
     static constexpr int kMergeFloats = (NKG - 1) * NMT * 16 * kMergeStride;
     static constexpr int kMergeMLFloats = (NKG - 1) * NMT * 16 * 2;
@@ -233,12 +236,25 @@ __device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t base, int row, int 
     return base + (uint32_t)((chunk >> 3) * kHalfBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
+// Same for an fp8 tile: one 128-byte row per key, 16-byte chunks 0..7 swizzled the same way.
+__device__ __forceinline__ uint32_t tile8_chunk_addr(uint32_t base, int row, int chunk) {
+    return base + (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
 // ---------------------------------------------------------------------------------------------
-template <int SRC, int NMT, int NKG, int NSTAGE, int MINB>
+// KV8 = true: K and V are fp8 (E4M3) codes, one 128-byte row per key and head, scaled by the
+// key and value scales (the key scale folded into scale_log2).  The tiles stream at half the
+// bytes; consumers widen them to fp16 in registers (exact) and run fp16 MMAs, with Q widened to
+// fp16 as well.  QK^T: ldmatrix on the fp8 tile hands each thread four consecutive dims of one
+// key, so the MMA's k index is permuted consistently in Q (loaded in the same order) and K.
+// PV: the widened V fragments are transposed in registers (movmatrix), which permutes the
+// output's head dims in a fixed way that the final store undoes.
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false>
 __global__ void __launch_bounds__((NMT * NKG + 1) * 32, MINB)
 attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const AttnArgs a) {
-    using L = SmemLayout<NMT, NKG, NSTAGE>;
+    using L = SmemLayout<NMT, NKG, NSTAGE, KV8>;
+    constexpr int kStage = KV8 ? kStageBytes8 : kStageBytes;
     constexpr int NWC = NMT * NKG;            // consumer warps
     constexpr int KPW = kTileKeys / NKG;      // keys per consumer warp per tile
     constexpr int NT = KPW / 8;               // S n-tiles per warp
@@ -310,8 +326,12 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 const uint32_t phase = (it / NSTAGE) & 1u;
                 if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) break;
                 meta[stage] = m;
-                uint8_t* st = smem + (size_t)stage * kStageBytes;
-                if (m.nvalid > 0) {
+                uint8_t* st = smem + (size_t)stage * kStage;
+                if (m.nvalid > 0 && KV8) {
+                    mbar_arrive_expect_tx(&full_bar[stage], kStageBytes8);
+                    tma_load_3d(st, &kmap, &full_bar[stage], 0, ty, tz, pol);
+                    tma_load_3d(st + kTileBytes8, &vmap, &full_bar[stage], 0, ty, tz, pol);
+                } else if (m.nvalid > 0) {
                     mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
                     tma_load_3d(st, &kmap, &full_bar[stage], 0, ty, tz, pol);
                     tma_load_3d(st + kHalfBytes, &kmap, &full_bar[stage], 64, ty, tz, pol);
@@ -344,6 +364,11 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     int row_ok[2];
     int Lpre = 0;
 
+    // head dim of accumulator pair (o[n][0], o[n][1]): 8 n + 2 tig; with fp8 KV the transposed
+    // V fragments put n-tile 2 j + h at dims 16 j + 4 tig + 2 h
+    auto out_dim = [](int n, int tg) -> int {
+        return KV8 ? 16 * (n >> 1) + 4 * tg + 2 * (n & 1) : 8 * n + 2 * tg;
+    };
     // per-lane ldmatrix row/chunk offsets
     const int k_row_l = (lane & 7) + ((lane >> 4) << 3);   // K: matrices (n0,k0) (n0,k8) (n8,k0) (n8,k8)
     const int k_chk_l = (lane >> 3) & 1;
@@ -390,32 +415,68 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 q32[r] = reinterpret_cast<const uint32_t*>(
                     a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD);
             }
+            if (KV8) {
+                // fp16 A-fragments with the k order of the fp8 K fragments: k slots (2 tig, +1)
+                // and (2 tig + 8, +9) of step ks hold dims 16 ks + 4 tig + (0, 1) and (2, 3)
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const int c = ks * 8 + tig;     // 32-bit word index of dims (16 ks + 2 tig)
-                qa[ks][0] = row_ok[0] ? __ldg(q32[0] + c) : 0u;
-                qa[ks][1] = row_ok[1] ? __ldg(q32[1] + c) : 0u;
-                qa[ks][2] = row_ok[0] ? __ldg(q32[0] + c + 4) : 0u;
-                qa[ks][3] = row_ok[1] ? __ldg(q32[1] + c + 4) : 0u;
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int c = ks * 8 + 2 * tig;
+                    qa[ks][0] = row_ok[0] ? bf16x2_to_f16x2(__ldg(q32[0] + c)) : 0u;
+                    qa[ks][1] = row_ok[1] ? bf16x2_to_f16x2(__ldg(q32[1] + c)) : 0u;
+                    qa[ks][2] = row_ok[0] ? bf16x2_to_f16x2(__ldg(q32[0] + c + 1)) : 0u;
+                    qa[ks][3] = row_ok[1] ? bf16x2_to_f16x2(__ldg(q32[1] + c + 1)) : 0u;
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int c = ks * 8 + tig;     // 32-bit word index of dims (16 ks + 2 tig)
+                    qa[ks][0] = row_ok[0] ? __ldg(q32[0] + c) : 0u;
+                    qa[ks][1] = row_ok[1] ? __ldg(q32[1] + c) : 0u;
+                    qa[ks][2] = row_ok[0] ? __ldg(q32[0] + c + 4) : 0u;
+                    qa[ks][3] = row_ok[1] ? __ldg(q32[1] + c + 4) : 0u;
+                }
             }
         }
 
         if (m.nvalid > 0) {
-            const uint32_t kbase = smem_addr(smem + (size_t)stage * kStageBytes);
-            const uint32_t vbase = kbase + kTileBytes;
+            const uint32_t kbase = smem_addr(smem + (size_t)stage * kStage);
+            const uint32_t vbase = kbase + (KV8 ? kTileBytes8 : kTileBytes);
             // ---- S = Q K^T over this warp's KPW keys -------------------------------------
             float s[NT][4];
 #pragma unroll
             for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+            if (KV8) {
+                // matrix (lane / 8): key octet 2 np + (lane / 8) % 2, dim chunk 2 kp + lane / 16
+                const int r8 = (lane & 7) + (((lane >> 3) & 1) << 3);
+                const int c8 = lane >> 4;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
+                for (int kp = 0; kp < 4; ++kp) {
 #pragma unroll
-                for (int np = 0; np < NT / 2; ++np) {
-                    uint32_t b0a, b1a, b0b, b1b;
-                    ldsm_x4(tile_chunk_addr(kbase, key0 + np * 16 + k_row_l, ks * 2 + k_chk_l),
-                            b0a, b1a, b0b, b1b);
-                    mma_bf16_16816(s[2 * np], qa[ks], b0a, b1a);
-                    mma_bf16_16816(s[2 * np + 1], qa[ks], b0b, b1b);
+                    for (int np = 0; np < NT / 2; ++np) {
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4(tile8_chunk_addr(kbase, key0 + np * 16 + r8, 2 * kp + c8), r0, r1, r2, r3);
+                        uint32_t b[8];
+                        e4m3x4_to_f16x2x2(r0, b[0], b[1]);
+                        e4m3x4_to_f16x2x2(r1, b[2], b[3]);
+                        e4m3x4_to_f16x2x2(r2, b[4], b[5]);
+                        e4m3x4_to_f16x2x2(r3, b[6], b[7]);
+                        mma_f16_16816(s[2 * np], qa[2 * kp], b[0], b[1]);
+                        mma_f16_16816(s[2 * np + 1], qa[2 * kp], b[2], b[3]);
+                        mma_f16_16816(s[2 * np], qa[2 * kp + 1], b[4], b[5]);
+                        mma_f16_16816(s[2 * np + 1], qa[2 * kp + 1], b[6], b[7]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        uint32_t b0a, b1a, b0b, b1b;
+                        ldsm_x4(tile_chunk_addr(kbase, key0 + np * 16 + k_row_l, ks * 2 + k_chk_l),
+                                b0a, b1a, b0b, b1b);
+                        mma_bf16_16816(s[2 * np], qa[ks], b0a, b1a);
+                        mma_bf16_16816(s[2 * np + 1], qa[ks], b0b, b1b);
+                    }
                 }
             }
             // ---- mask: ragged tile end, in-step (causal / tree) keys ----------------------
@@ -466,9 +527,17 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 for (int n = 0; n < NT; ++n) {
                     const float p0 = fast_exp2(fmaf(s[n][2 * r], a.scale_log2, -m_use[r]));
                     const float p1 = fast_exp2(fmaf(s[n][2 * r + 1], a.scale_log2, -m_use[r]));
-                    const uint32_t pk = pack_bf16x2(p0, p1);
-                    // the row sum uses the same bf16-rounded weights the PV product uses
-                    l_r[r] += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+                    uint32_t pk;
+                    if (KV8) {
+                        // fp16 weights; the row sum uses the same rounded weights
+                        pk = pack_f16x2(p0, p1);
+                        const float2 pr = __half22float2(*reinterpret_cast<const __half2*>(&pk));
+                        l_r[r] += pr.x + pr.y;
+                    } else {
+                        pk = pack_bf16x2(p0, p1);
+                        // the row sum uses the same bf16-rounded weights the PV product uses
+                        l_r[r] += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+                    }
                     pa[n >> 1][r + 2 * (n & 1)] = pk;
                 }
             }
@@ -483,17 +552,47 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     lo_keep = (k0 < m.nvalid ? 0x0000ffffu : 0u) | (k0 + 1 < m.nvalid ? 0xffff0000u : 0u);
                     hi_keep = (k0 + 8 < m.nvalid ? 0x0000ffffu : 0u) | (k0 + 9 < m.nvalid ? 0xffff0000u : 0u);
                 }
+                if (KV8) {
+                    // matrix (lane / 8): key octet (lane / 8) % 2, dim chunk 2 jp + lane / 16.
+                    // Widened, each matrix is two 8x8 fp16 matrices (dims 16 j + 4 c + {0, 1} and
+                    // + {2, 3}); transposed, they are the B fragments of output tiles 2 j, 2 j + 1.
+                    const int r8 = (lane & 7) + (((lane >> 3) & 1) << 3);
+                    const int c8 = lane >> 4;
 #pragma unroll
-                for (int dp = 0; dp < 8; ++dp) {
-                    uint32_t b0a, b1a, b0b, b1b;
-                    ldsm_x4_trans(tile_chunk_addr(vbase, krow + v_row_l, dp * 2 + v_chk_l),
-                                  b0a, b1a, b0b, b1b);
-                    if (ragged) {
-                        b0a &= lo_keep; b0b &= lo_keep;
-                        b1a &= hi_keep; b1b &= hi_keep;
+                    for (int jp = 0; jp < 4; ++jp) {
+                        uint32_t r[4];
+                        ldsm_x4(tile8_chunk_addr(vbase, krow + r8, 2 * jp + c8), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int j = 2 * jp + h;
+                            uint32_t x00, x01, x10, x11;
+                            e4m3x4_to_f16x2x2(r[2 * h], x00, x01);
+                            e4m3x4_to_f16x2x2(r[2 * h + 1], x10, x11);
+                            uint32_t b00 = movmatrix_trans(x00);
+                            uint32_t b10 = movmatrix_trans(x10);
+                            uint32_t b01 = movmatrix_trans(x01);
+                            uint32_t b11 = movmatrix_trans(x11);
+                            if (ragged) {
+                                b00 &= lo_keep; b01 &= lo_keep;
+                                b10 &= hi_keep; b11 &= hi_keep;
+                            }
+                            mma_f16_16816(o[2 * j], pa[kk], b00, b10);
+                            mma_f16_16816(o[2 * j + 1], pa[kk], b01, b11);
+                        }
                     }
-                    mma_bf16_16816(o[2 * dp], pa[kk], b0a, b1a);
-                    mma_bf16_16816(o[2 * dp + 1], pa[kk], b0b, b1b);
+                } else {
+#pragma unroll
+                    for (int dp = 0; dp < 8; ++dp) {
+                        uint32_t b0a, b1a, b0b, b1b;
+                        ldsm_x4_trans(tile_chunk_addr(vbase, krow + v_row_l, dp * 2 + v_chk_l),
+                                      b0a, b1a, b0b, b1b);
+                        if (ragged) {
+                            b0a &= lo_keep; b0b &= lo_keep;
+                            b1a &= hi_keep; b1b &= hi_keep;
+                        }
+                        mma_bf16_16816(o[2 * dp], pa[kk], b0a, b1a);
+                        mma_bf16_16816(o[2 * dp + 1], pa[kk], b0b, b1b);
+                    }
                 }
             }
         }
@@ -556,7 +655,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     const int rr = mt * 16 + gid + 8 * r;            // row within the block
                     const int R = m.rb * kRowsPerBlock + rr;
                     const float l = l_r[r];
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    const float inv = l > 0.f ? a.v_scale / l : 0.f;
                     const float lse2 = l > 0.f ? m_r[r] + __log2f(l) : -INFINITY;
                     if (m.flags & kWhole) {
                         const int i = R / a.G, g = R - (R / a.G) * a.G;
@@ -564,13 +663,13 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         uint32_t* op = reinterpret_cast<uint32_t*>(a.out + orow * kD);
 #pragma unroll
                         for (int n = 0; n < 16; ++n)
-                            op[n * 4 + tig] = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+                            op[out_dim(n, tig) >> 1] = pack_bf16x2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
                         if (a.lse != nullptr && tig == 0) a.lse[orow] = lse2 * kLn2;
                     } else {
                         float* wo = a.ws_o + ((size_t)slot * a.rows_blk + rr) * kD;
 #pragma unroll
                         for (int n = 0; n < 16; ++n)
-                            *reinterpret_cast<float2*>(wo + n * 8 + 2 * tig) =
+                            *reinterpret_cast<float2*>(wo + out_dim(n, tig)) =
                                 make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
                         if (tig == 0) a.ws_lse[(size_t)slot * a.rows_blk + rr] = lse2;
                     }

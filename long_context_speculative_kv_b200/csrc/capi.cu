@@ -83,16 +83,20 @@ int encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 }
 
 // A [n_blocks][rows][128] bf16 tensor viewed as 3-D (dim, row, block), read in 64x64 boxes with
-// the 128-byte swizzle.  Rows past `rows` and blocks past `n_blocks` read as zero.
-int encode_rows_map(CUtensorMap* map, const void* base, long long rows, long long n_blocks) {
+// the 128-byte swizzle.  Rows past `rows` and blocks past `n_blocks` read as zero.  fp8: the
+// same with 1-byte elements, read in 128x64 boxes (one 128-byte row per key).
+int encode_rows_map(CUtensorMap* map, const void* base, long long rows, long long n_blocks,
+                    bool fp8 = false) {
     PFN_cuTensorMapEncodeTiled_v12000 enc;
     int rc = encoder(&enc);
     if (rc != WMTP_OK) return rc;
+    const cuuint64_t esz = fp8 ? 1 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)n_blocks};
-    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * esz, (cuuint64_t)rows * kD * esz};
+    cuuint32_t box[3] = {fp8 ? 128u : 64u, (cuuint32_t)kTileKeys, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+    CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
@@ -207,11 +211,11 @@ char variant_for(int nmt) {
     return v[nmt];
 }
 
-template <int SRC, int NMT, int NKG, int NSTAGE, int MINB>
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false>
 int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                   const Shape& s, cudaStream_t st) {
-    using Lay = SmemLayout<NMT, NKG, NSTAGE>;
-    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB>;
+    using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8>;
+    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB, KV8>;
     static bool attr_set[kMaxDevices] = {};
     int dev;
     if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
@@ -289,9 +293,25 @@ int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, 
     }
 }
 
+// fp8-KV layouts per m-tile count (key groups, stages of 16 KiB, CTAs per SM), two CTAs per SM
+// throughout: widening the codes lengthens each warp's dependency chains, so the consumer warps
+// need the second CTA's warps to hide them (ncu on the one-CTA layout: 5 warps per SM, issue
+// slots 32 % busy, stalls mostly on fixed-latency dependencies).
+template <int SRC>
+int launch_attn_kv8(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
+                    const Shape& s, cudaStream_t st) {
+    switch ((s.rows_blk + 15) / 16) {
+        case 1: return launch_attn_t<SRC, 1, 4, 4, 2, true>(km, vm, a, sm_count, s, st);
+        case 2: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
+        case 3: return launch_attn_t<SRC, 3, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
+        default: return launch_attn_t<SRC, 4, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
+    }
+}
+
 template <int SRC>
 int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
-                const Shape& s, cudaStream_t st) {
+                const Shape& s, cudaStream_t st, bool kv8 = false) {
+    if (kv8) return launch_attn_kv8<SRC>(km, vm, a, sm_count, s, st);
     if (use_tc(s)) return launch_attn_tc<SRC>(km, vm, a.q, a, sm_count, s, st);
     const int nmt = (s.rows_blk + 15) / 16;
     switch (nmt) {
@@ -323,7 +343,8 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
 }
 
 // CTAs per SM of the variant a call with these rows will use.
-int ctas_per_sm_for(const Shape& s) {
+int ctas_per_sm_for(const Shape& s, bool kv8 = false) {
+    if (kv8) return 2;
     if (use_tc(s)) return tc_ctas_per_sm();
     const int nmt = (s.rows_blk + 15) / 16;
     const char v = variant_for(nmt < 4 ? nmt : 4);
@@ -334,14 +355,18 @@ int ctas_per_sm_for(const Shape& s) {
 
 // Common front half of the three attention calls.
 int prepare(const Shape& s, const void* q, const void* out, const float* lse, void* ws,
-            size_t ws_bytes, float sm_scale, DeviceInfo* dev, AttnArgs* a) {
+            size_t ws_bytes, float sm_scale, DeviceInfo* dev, AttnArgs* a, bool kv8 = false,
+            float k_scale = 1.f, float v_scale = 1.f) {
     if (q == nullptr || out == nullptr || ws == nullptr) return WMTP_ERR_ARG;
     if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return WMTP_ERR_ARG;
+    if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+        return WMTP_ERR_ARG;
+    if (!std::isfinite(sm_scale * k_scale * 1.4426950408889634f)) return WMTP_ERR_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || (lse && !aligned(lse, 4)) || !aligned(ws, 256))
         return WMTP_ERR_ALIGN;
     int rc = device_info(dev);
     if (rc != WMTP_OK) return rc;
-    const long long slots = (long long)dev->sm_count * ctas_per_sm_for(s) + s.units;
+    const long long slots = (long long)dev->sm_count * ctas_per_sm_for(s, kv8) + s.units;
     if (ws_bytes < ws_total_bytes(slots, s.rows_blk)) return WMTP_ERR_WORKSPACE;
     std::memset(a, 0, sizeof(*a));
     a->q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -353,16 +378,17 @@ int prepare(const Shape& s, const void* q, const void* out, const float* lse, vo
     a->B = s.B; a->n_q = s.n_q; a->Hq = s.Hq; a->Hkv = s.Hkv; a->G = s.G; a->n_rb = s.n_rb;
     a->rows_total = s.rows_total;
     a->rows_blk = s.rows_blk;
-    a->scale_log2 = sm_scale * 1.4426950408889634f;
+    a->scale_log2 = sm_scale * k_scale * 1.4426950408889634f;
+    a->v_scale = v_scale;
     a->min_tiles_per_cta = min_tiles_per_cta();
     return WMTP_OK;
 }
 
-int paged_call(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_pool,
+int paged_call(const wmtp_bf16* q, const void* k_pool, const void* v_pool,
                const int32_t* page_table, const int32_t* kv_len, const int32_t* tree_parent,
                int B, int n_q, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages,
                float sm_scale, wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
-               cudaStream_t st) {
+               cudaStream_t st, bool kv8 = false, float k_scale = 1.f, float v_scale = 1.f) {
     Shape s;
     int rc = check_shape(B, n_q, Hq, Hkv, D, &s);
     if (rc != WMTP_OK) return rc;
@@ -376,7 +402,7 @@ int paged_call(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_p
         return WMTP_ERR_ALIGN;
     DeviceInfo dev;
     AttnArgs a;
-    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a);
+    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a, kv8, k_scale, v_scale);
     if (rc != WMTP_OK) return rc;
     a.tree_parent = tree_parent;
     a.page_table = page_table;
@@ -384,9 +410,9 @@ int paged_call(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_p
     a.max_pages = max_pages;
     a.num_pages = num_pages;
     CUtensorMap km, vm;
-    if ((rc = encode_rows_map(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
-    if ((rc = encode_rows_map(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
-    return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st);
+    if ((rc = encode_rows_map(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv, kv8)) != WMTP_OK) return rc;
+    if ((rc = encode_rows_map(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv, kv8)) != WMTP_OK) return rc;
+    return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st, kv8);
 }
 
 }  // namespace
@@ -449,9 +475,16 @@ size_t wmtp_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D) {
     return ws_total_bytes((long long)dev.sm_count * kMaxCtasPerSm + s.units, s.rows_blk);
 }
 
-int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, const wmtp_bf16* k_new,
-                   const wmtp_bf16* v_new, int B, int n_new, int Hkv, int D, int n_sink, int capacity,
-                   wmtp_stream_t stream) {
+}  // extern "C"
+
+namespace wmtp {
+namespace {
+
+// Ring append of rows of CH 16-byte pieces (bf16: 16, fp8: 8).
+template <int CH>
+int ring_append_call(void* ring_k, void* ring_v, int64_t* ring_len, const void* k_new,
+                     const void* v_new, int B, int n_new, int Hkv, int D, int n_sink, int capacity,
+                     wmtp_stream_t stream) {
     if (ring_k == nullptr || ring_v == nullptr || ring_len == nullptr) return WMTP_ERR_ARG;
     if (B < 1 || n_new < 0 || Hkv < 1 || n_sink < 0 || capacity <= n_sink) return WMTP_ERR_ARG;
     if (D != WMTP_HEAD_DIM) return WMTP_ERR_SHAPE;
@@ -467,13 +500,13 @@ int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, cons
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // upper bound on surviving rows per request: the sink plus the ring's other slots
     const long long surv = (long long)(n_new < capacity ? n_new : capacity);
-    const long long work = surv * Hkv * 16;
+    const long long work = surv * Hkv * CH;
     long long chunks = (work + 256 * 4 - 1) / (256 * 4);     // ~4 pieces per thread
     const long long max_chunks = (long long)dev.sm_count * 8;
     if (chunks > max_chunks) chunks = max_chunks;
     if (chunks < 1) chunks = 1;
     const int single = (chunks == 1);
-    rc = launch(ring_append_kernel, dim3((unsigned)chunks, B), dim3(256), 0, st,
+    rc = launch(ring_append_kernel<CH>, dim3((unsigned)chunks, B), dim3(256), 0, st,
                 reinterpret_cast<uint4*>(ring_k), reinterpret_cast<uint4*>(ring_v),
                 reinterpret_cast<long long*>(ring_len), reinterpret_cast<const uint4*>(k_new),
                 reinterpret_cast<const uint4*>(v_new), n_new, Hkv, n_sink, capacity, single);
@@ -482,10 +515,10 @@ int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, cons
                   reinterpret_cast<long long*>(ring_len), B, n_new);
 }
 
-int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,
-                      const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D, int n_sink,
-                      int window, int capacity, float sm_scale, wmtp_bf16* out, float* lse, void* ws,
-                      size_t ws_bytes, wmtp_stream_t stream) {
+int window_call(const wmtp_bf16* q, const void* ring_k, const void* ring_v, const int64_t* ring_len,
+                int B, int n_q, int Hq, int Hkv, int D, int n_sink, int window, int capacity,
+                float sm_scale, wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                wmtp_stream_t stream, bool kv8, float k_scale, float v_scale) {
     Shape s;
     int rc = check_shape(B, n_q, Hq, Hkv, D, &s);
     if (rc != WMTP_OK) return rc;
@@ -495,16 +528,71 @@ int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf
     if (!aligned(ring_k, 16) || !aligned(ring_v, 16) || !aligned(ring_len, 8)) return WMTP_ERR_ALIGN;
     DeviceInfo dev;
     AttnArgs a;
-    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a);
+    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a, kv8, k_scale, v_scale);
     if (rc != WMTP_OK) return rc;
     a.ring_len = reinterpret_cast<const long long*>(ring_len);
     a.n_sink = n_sink;
     a.window = window;
     a.capacity = capacity;
     CUtensorMap km, vm;
-    if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
-    if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
-    return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, reinterpret_cast<cudaStream_t>(stream));
+    if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
+    if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
+    return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, reinterpret_cast<cudaStream_t>(stream), kv8);
+}
+
+}  // namespace
+}  // namespace wmtp
+
+extern "C" {
+
+int ring_kv_append(wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len, const wmtp_bf16* k_new,
+                   const wmtp_bf16* v_new, int B, int n_new, int Hkv, int D, int n_sink, int capacity,
+                   wmtp_stream_t stream) {
+    return wmtp::ring_append_call<16>(ring_k, ring_v, ring_len, k_new, v_new, B, n_new, Hkv, D, n_sink,
+                                      capacity, stream);
+}
+
+int ring_kv_append_fp8(uint8_t* ring_k, uint8_t* ring_v, int64_t* ring_len, const uint8_t* k_new,
+                       const uint8_t* v_new, int B, int n_new, int Hkv, int D, int n_sink, int capacity,
+                       wmtp_stream_t stream) {
+    return wmtp::ring_append_call<8>(ring_k, ring_v, ring_len, k_new, v_new, B, n_new, Hkv, D, n_sink,
+                                     capacity, stream);
+}
+
+int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf16* ring_v,
+                      const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D, int n_sink,
+                      int window, int capacity, float sm_scale, wmtp_bf16* out, float* lse, void* ws,
+                      size_t ws_bytes, wmtp_stream_t stream) {
+    return window_call(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
+                       sm_scale, out, lse, ws, ws_bytes, stream, false, 1.f, 1.f);
+}
+
+int draft_attn_window_fp8(const wmtp_bf16* q, const uint8_t* ring_k, const uint8_t* ring_v,
+                          const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D, int n_sink,
+                          int window, int capacity, float sm_scale, float k_scale, float v_scale,
+                          wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes, wmtp_stream_t stream) {
+    return window_call(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
+                       sm_scale, out, lse, ws, ws_bytes, stream, true, k_scale, v_scale);
+}
+
+int draft_attn_full_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const uint8_t* v_pool,
+                        const int32_t* page_table, const int32_t* kv_len, int B, int n_q, int Hq, int Hkv,
+                        int D, int page_size, int max_pages, int num_pages, float sm_scale, float k_scale,
+                        float v_scale, wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                        wmtp_stream_t stream) {
+    return paged_call(q, k_pool, v_pool, page_table, kv_len, nullptr, B, n_q, Hq, Hkv, D, page_size,
+                      max_pages, num_pages, sm_scale, out, lse, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), true, k_scale, v_scale);
+}
+
+int verify_attn_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const uint8_t* v_pool,
+                    const int32_t* page_table, const int32_t* kv_len, const int32_t* tree_parent, int B,
+                    int n_q, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages,
+                    float sm_scale, float k_scale, float v_scale, wmtp_bf16* out, float* lse, void* ws,
+                    size_t ws_bytes, wmtp_stream_t stream) {
+    return paged_call(q, k_pool, v_pool, page_table, kv_len, tree_parent, B, n_q, Hq, Hkv, D, page_size,
+                      max_pages, num_pages, sm_scale, out, lse, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), true, k_scale, v_scale);
 }
 
 int draft_attn_full(const wmtp_bf16* q, const wmtp_bf16* k_pool, const wmtp_bf16* v_pool,

@@ -4,6 +4,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -146,6 +148,44 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------------------------------------
+// fp16 MMA and fp8 (E4M3) widening, for the fp8-KV path: every E4M3 value and every bf16 query
+// of normal magnitude is exact in fp16, so the products see the stored numbers unrounded.
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Four E4M3 codes (a 32-bit word, lowest byte first) -> two fp16x2 words: lo = codes 0, 1 and
+// hi = codes 2, 3 (the lower code in the lower half), with one cvt per pair.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 c01, c23;\n\t"
+        "mov.b32 {c01, c23}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
+        : "=r"(lo), "=r"(hi) : "r"(codes));
+}
+
+// bf16x2 -> fp16x2 through fp32 (exact for values fp16 represents).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Transposes the 8x8 16-bit matrix a warp holds in the ldmatrix fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

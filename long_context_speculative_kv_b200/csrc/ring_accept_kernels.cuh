@@ -12,11 +12,13 @@ namespace wmtp {
 // Of the call's positions [L_old, L_new) only the survivors are copied: the sink positions
 // (p < n_sink) and the last C - n_sink positions; an earlier position that a later one of the
 // same call would overwrite is never written, so no two threads write one slot.
-// Grid (chunks, B), 256 threads; each thread moves 16-byte pieces of 256-byte rows.
+// Grid (chunks, B), 256 threads; each thread moves 16-byte pieces of rows of CH pieces (16 for
+// bf16 rows of 256 bytes, 8 for fp8 rows of 128 bytes).
 __device__ __forceinline__ long long ring_slot_of(long long p, int s, int C) {
     return p < s ? p : (long long)s + (p - s) % (long long)(C - s);
 }
 
+template <int CH>
 __global__ void __launch_bounds__(256)
 ring_append_kernel(uint4* __restrict__ ring_k, uint4* __restrict__ ring_v, long long* ring_len,
                    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
@@ -32,7 +34,7 @@ ring_append_kernel(uint4* __restrict__ ring_k, uint4* __restrict__ ring_v, long 
     long long s2 = (long long)n_new - (C - n_sink);
     if (s2 < e1) s2 = e1;
     const long long n_surv = e1 + (n_new - s2);
-    constexpr int kChunks = 256 / 16;                        // 16-byte pieces per row
+    constexpr int kChunks = CH;                              // 16-byte pieces per row
     const long long work = n_surv * Hkv * kChunks;
     for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < work;
          w += (long long)gridDim.x * blockDim.x) {

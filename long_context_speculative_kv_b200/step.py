@@ -56,6 +56,10 @@ class StepBuffers:
     kv_len_ctx: Optional[torch.Tensor] = None
     kv_len_fwd: Optional[List[torch.Tensor]] = None
     sm_scale: float = 128 ** -0.5
+    # fp8 (E4M3) KV: every K/V cache and new row holds codes, scaled by k_scale / v_scale
+    kv8: bool = False
+    k_scale: float = 1.0
+    v_scale: float = 1.0
     # outputs / workspace
     ws: Optional[torch.Tensor] = None
     out: Dict[str, torch.Tensor] = field(default_factory=dict)
@@ -108,34 +112,59 @@ class DecodeStep:
     def draft_windowed(self, log: Optional[CallLog] = None):
         b = self.b
         if log: log.mark("append_ctx")
-        api.ring_kv_append(b.ring_k, b.ring_v, b.ring_len, b.k_ctx, b.v_ctx, b.n_sink)
+        self._append(b.k_ctx, b.v_ctx)
         if log: log.mark("window_ctx")
-        api.draft_attn_window(b.q_ctx, b.ring_k, b.ring_v, b.ring_len, b.n_sink, b.window, b.sm_scale,
-                              b.ws, out=b.out["ctx"], lse=b.out["ctx_lse"])
+        self._window(b.q_ctx, b.out["ctx"], b.out["ctx_lse"])
         for j in range(self.gamma):
             if log: log.mark("append_fwd")
-            api.ring_kv_append(b.ring_k, b.ring_v, b.ring_len, b.k_fwd[j], b.v_fwd[j], b.n_sink)
+            self._append(b.k_fwd[j], b.v_fwd[j])
             if log: log.mark("window_fwd")
-            api.draft_attn_window(b.q_fwd[j], b.ring_k, b.ring_v, b.ring_len, b.n_sink, b.window,
-                                  b.sm_scale, b.ws, out=b.out["fwd"], lse=b.out["fwd_lse"])
+            self._window(b.q_fwd[j], b.out["fwd"], b.out["fwd_lse"])
+
+    def _append(self, k_new, v_new):
+        b = self.b
+        if b.kv8:
+            api.ring_kv_append_fp8(b.ring_k, b.ring_v, b.ring_len, k_new, v_new, b.n_sink)
+        else:
+            api.ring_kv_append(b.ring_k, b.ring_v, b.ring_len, k_new, v_new, b.n_sink)
+
+    def _window(self, q, out, lse):
+        b = self.b
+        if b.kv8:
+            api.draft_attn_window_fp8(q, b.ring_k, b.ring_v, b.ring_len, b.n_sink, b.window, b.sm_scale,
+                                      b.k_scale, b.v_scale, b.ws, out=out, lse=lse)
+        else:
+            api.draft_attn_window(q, b.ring_k, b.ring_v, b.ring_len, b.n_sink, b.window, b.sm_scale,
+                                  b.ws, out=out, lse=lse)
+
+    def _full(self, q, kv_len, out, lse):
+        b = self.b
+        if b.kv8:
+            api.draft_attn_full_fp8(q, b.k_draft, b.v_draft, b.table_d, kv_len, b.sm_scale, b.k_scale,
+                                    b.v_scale, b.ws, out=out, lse=lse)
+        else:
+            api.draft_attn_full(q, b.k_draft, b.v_draft, b.table_d, kv_len, b.sm_scale, b.ws, out=out, lse=lse)
 
     def draft_native(self, log: Optional[CallLog] = None):
         b = self.b
         if log: log.mark("full_ctx")
-        api.draft_attn_full(b.q_ctx, b.k_draft, b.v_draft, b.table_d, b.kv_len_ctx, b.sm_scale, b.ws,
-                            out=b.out["ctx"], lse=b.out["ctx_lse"])
+        self._full(b.q_ctx, b.kv_len_ctx, b.out["ctx"], b.out["ctx_lse"])
         for j in range(self.gamma):
             if log: log.mark("full_fwd")
-            api.draft_attn_full(b.q_fwd[j], b.k_draft, b.v_draft, b.table_d, b.kv_len_fwd[j],
-                                b.sm_scale, b.ws, out=b.out["fwd"], lse=b.out["fwd_lse"])
+            self._full(b.q_fwd[j], b.kv_len_fwd[j], b.out["fwd"], b.out["fwd_lse"])
 
     def verify(self, log: Optional[CallLog] = None):
         b = self.b
         for layer in range(self.n_layers):
             if log: log.mark("verify")
-            api.verify_attn(b.q_verify[layer], b.k_pools[layer], b.v_pools[layer], b.table_v,
-                            b.kv_len_v, b.sm_scale, b.ws, tree_parent=b.tree_parent,
-                            out=b.out["verify"], lse=b.out["verify_lse"])
+            if b.kv8:
+                api.verify_attn_fp8(b.q_verify[layer], b.k_pools[layer], b.v_pools[layer], b.table_v,
+                                    b.kv_len_v, b.sm_scale, b.k_scale, b.v_scale, b.ws,
+                                    tree_parent=b.tree_parent, out=b.out["verify"], lse=b.out["verify_lse"])
+            else:
+                api.verify_attn(b.q_verify[layer], b.k_pools[layer], b.v_pools[layer], b.table_v,
+                                b.kv_len_v, b.sm_scale, b.ws, tree_parent=b.tree_parent,
+                                out=b.out["verify"], lse=b.out["verify_lse"])
 
     def accept(self, log: Optional[CallLog] = None):
         b = self.b

@@ -129,3 +129,16 @@ def host_head_sequence(tok: torch.Tensor, b: int, h: int, L: int) -> np.ndarray:
     """bf16 bits [1, 1, L, D] of request b, kv head h, from a token-major device tensor."""
     seq = tok[b, :L, h].contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
     return seq.reshape(1, 1, L, -1)
+
+
+def kv_rows_fp8(shape, g: torch.Generator, device, scale: float = 2.0):
+    """K and V of ``shape`` as E4M3 codes (uint8): N(0, scale^2) rounded to the nearest code."""
+    k = torch.empty(shape, dtype=torch.uint8, device=device)
+    v = torch.empty(shape, dtype=torch.uint8, device=device)
+    for t in (k, v):
+        flat = t.view(-1)
+        for s in range(0, flat.numel(), CHUNK):
+            n = min(CHUNK, flat.numel() - s)
+            x = torch.randn(n, generator=g, device=device, dtype=torch.float32).mul_(scale)
+            flat[s:s + n].copy_(x.to(torch.float8_e4m3fn).view(torch.uint8))
+    return k, v

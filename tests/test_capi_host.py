@@ -29,7 +29,8 @@ def test_header_declares_the_five_calls_and_helpers():
     assert {"ring_kv_append", "draft_attn_window", "draft_attn_full", "verify_attn",
             "accept_greedy", "wmtp_workspace_bytes", "wmtp_status_string",
             "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc",
-            "accept_stochastic", "ring_kv_append_at", "spec_commit", "wmtp_synth_draft_tokens",
+            "accept_stochastic", "ring_kv_append_at", "spec_commit", "ring_kv_append_fp8",
+            "draft_attn_window_fp8", "draft_attn_full_fp8", "verify_attn_fp8", "wmtp_synth_draft_tokens",
             "wmtp_synth_target_logits"} == names
     assert set(_lib._SIGNATURES) == names
 
@@ -99,6 +100,21 @@ def test_accept_host_checks(lib):
     assert a(GOOD, GOOD, None, 1, 65, 1024, GOOD, GOOD, None) == -1
     assert a(GOOD, GOOD, None, 1, 4, 0, GOOD, GOOD, None) == -1
     assert a(ctypes.c_void_p(0x10002), GOOD, None, 1, 4, 1024, GOOD, GOOD, None) == -3
+
+
+def test_fp8_host_checks(lib):
+    w = lib.draft_attn_window_fp8
+    # (q, rk, rv, rlen, B, n_q, Hq, Hkv, D, s, W, C, scale, k_scale, v_scale, out, lse, ws, n, stream)
+    assert w(GOOD, GOOD, GOOD, GOOD, 1, 1, 8, 2, 128, 4, 252, 256, 1.0, 0.0, 1.0, GOOD, None, GOOD, 1 << 30, None) == -1
+    assert w(GOOD, GOOD, GOOD, GOOD, 1, 1, 8, 2, 128, 4, 252, 256, 1.0, 1.0, float("inf"), GOOD, None, GOOD, 1 << 30, None) == -1
+    assert w(GOOD, GOOD, GOOD, GOOD, 1, 1, 8, 3, 128, 4, 252, 256, 1.0, 1.0, 1.0, GOOD, None, GOOD, 1 << 30, None) == -2
+    f = lib.draft_attn_full_fp8
+    assert f(GOOD, GOOD, GOOD, GOOD, GOOD, 1, 1, 8, 2, 128, 32, 4, 4, 1.0, 1.0, 1.0, GOOD, None, GOOD, 1 << 30, None) == -2
+    v = lib.verify_attn_fp8
+    assert v(GOOD, GOOD, GOOD, GOOD, GOOD, BAD, 1, 4, 8, 2, 128, 64, 4, 4, 1.0, 1.0, 1.0, GOOD, None, GOOD, 1 << 30, None) == -3
+    r = lib.ring_kv_append_fp8
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, 1, 1, 2, 64, 4, 256, None) == -2
+    assert r(GOOD, GOOD, GOOD, GOOD, GOOD, 1, 0, 2, 128, 4, 256, None) == 0
 
 
 def test_stochastic_accept_host_checks(lib):
