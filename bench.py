@@ -59,6 +59,23 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of the ranks' values (every rank gets it); the identity on one rank."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_us_per_step(ms_max: float, steps: int, world: int) -> float:
+    """Whole-job time per decode step: N replicas ran steps x N steps in the slowest rank's
+    time (weak scaling, no exchange between replicas)."""
+    return ms_max * 1e3 / (steps * world)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -155,11 +172,7 @@ def run_gpu(args):
             dist.barrier()
 
     def max_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(x, world, device)
 
     w = configs.BY_NAME[args.workload]
     if args.context:
@@ -294,7 +307,7 @@ def run_gpu(args):
     us_w_local = ms_w * 1e3 / args.steps
     us_n_local = ms_n * 1e3 / args.steps
     ms_w_max, ms_n_max = max_ranks(ms_w), max_ranks(ms_n)
-    value = ms_w_max * 1e3 / (args.steps * world)          # aggregate: all ranks' steps
+    value = aggregate_us_per_step(ms_w_max, args.steps, world)
     tdw, tvw, taw = phases(logs_w, {"append_ctx", "window_ctx", "append_fwd", "window_fwd"})
     tdn, tvn, tan = phases(logs_n, {"full_ctx", "full_fwd"})
 
@@ -373,7 +386,7 @@ def run_gpu(args):
         ms_e2e = timed_graph(g_w, args.steps, e2e=(h_in, h_out))
     else:
         ms_e2e, _, _ = timed("windowed", args.steps, e2e=(h_in, h_out))
-    e2e_value = max_ranks(ms_e2e) * 1e3 / (args.steps * world)
+    e2e_value = aggregate_us_per_step(max_ranks(ms_e2e), args.steps, world)
     if use_graph:
         del g_w, g_n
 
