@@ -701,7 +701,20 @@ class OracleSample:
 
 
 def oracle_step_estimate(w, gamma, window, lens, n_q_v, n_layers):
-    return OracleSample(w, gamma, window, int(lens[0]), n_q_v, n_layers).estimate()
+    """The all-core estimate, plus the same verify sample on one core (the oracle's per-row
+    loop parallelises over rows, so the one-core figure scales the verify part)."""
+    smp = OracleSample(w, gamma, window, int(lens[0]), n_q_v, n_layers)
+    res = smp.estimate()
+    o = smp.oracle
+    rows = [(0, i % smp.n_q_v, (i // smp.n_q_v) % w.G) for i in range(4)]
+    t1 = smp._time(lambda: o.attention(smp.qv, smp.kv, smp.vv, [smp.Lv], o.MODE_CAUSAL, w.sm_scale,
+                                       rows=rows, n_threads=1))
+    t_verify_1 = t1 * smp.n_q_v * w.Hq * smp.n_layers * w.B / len(rows)
+    res["value_1_core"] = round((t_verify_1 + res["t_draft_windowed_us"] * 1e-6 * smp.cores
+                                 + res["t_accept_us"] * 1e-6) * 1e6, 1)
+    res["value_1_core_is"] = ("verify from 4 rows on one core; windowed draft scaled from the all-core "
+                              "time by the core count")
+    return res
 
 
 def run_reference(args):
