@@ -69,6 +69,7 @@ struct TileMeta {
     int nvalid;     // rows [0, nvalid) are keys of this unit; 0 = skipped tile
     int L_tot;      // request length (keys) including this call's n_q positions
     int flags;      // kFirst | kLast | kWhole
+    int ord;        // units this CTA finished before this tile's unit (tcgen05 kernel only)
 };
 enum : int { kFirst = 1, kLast = 2, kWhole = 4 };
 

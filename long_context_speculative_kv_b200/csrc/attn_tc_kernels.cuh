@@ -5,7 +5,7 @@
 // [128 x 64] contractions per key tile.
 //
 // Same work split, tile walk, masks, partial format and merge as attn_split_kernel; only the
-// math engine differs.  Roles (256 threads, one CTA per SM):
+// math engine differs.  Roles (384 threads, one CTA per SM):
 //   warp 0        K producer: each tile's K (two 64x64 TMA boxes) into an NK-deep ring, and each
 //                 unit's Q rows (one box of n_q x G rows per 64-dim half) into a Q double buffer;
 //   warp 6        V producer: each tile's V into an NV-deep ring.  K is released as soon as
@@ -17,17 +17,23 @@
 //   warp 7        lane 0 issues O += P V (M = 64, N = 128 dims, K = 64 keys; O stays in TMEM)
 //                 once the softmax warps have written P(t).  Two issuers keep the tensor core's
 //                 queue fed while the other waits;
-//   warps 2..5    softmax: the M = 64 accumulator keeps row r in TMEM lane 32 (r / 16) + r % 16,
-//                 so warp w sees rows 16 (w % 4) .. + 15; with the 16x32bx2 load both half-warps
-//                 read those rows, lanes 0-15 keys 0-31 and lanes 16-31 keys 32-63 (and O dims
-//                 0-63 / 64-127).  Each thread masks, exponentiates against the row's running
-//                 maximum and writes its half of the P row (bf16, 128-byte swizzled) for the PV
-//                 MMA.  The maximum is only moved when a row's maximum grows by more than 2^8
-//                 (log2 units), and only then is that O row rescaled in TMEM, so the common
-//                 tile touches no O at all.
-// Tensor memory: NSB S buffers of 64 columns, then O (128 columns).  Every wait is bounded; on a
-// timeout all roles stop, each MMA issuer waits (bounded) for its own MMAs, all meet at the final
-// barrier and warp 1 frees the tensor memory.
+//   warps 2..5, 8..11   softmax, two groups of four warps taking alternate tiles (group g the
+//                 CTA's tiles it with it % 2 == g), each with its own running maxima and sums and
+//                 its own O accumulator in TMEM; one warp per sub-partition could not keep up
+//                 with the tile rate.  The M = 64 accumulator keeps row r in TMEM lane
+//                 32 (r / 16) + r % 16, so warp w sees rows 16 (w % 4) .. + 15; with the 16x32bx2
+//                 load both half-warps read those rows, lanes 0-15 keys 0-31 and lanes 16-31
+//                 keys 32-63 (and O dims 0-63 / 64-127).  Each thread masks, exponentiates against
+//                 the row's running maximum and writes its half of the P row (bf16, 128-byte
+//                 swizzled) for the PV MMA.  The maximum is only moved when a row's maximum grows
+//                 by more than 2^8 (log2 units), and only then is that O row rescaled in TMEM, so
+//                 the common tile touches no O at all.  After each tile a group publishes its
+//                 rows' maxima and sums; the group holding a unit's last tile combines both
+//                 groups' (O, max, sum) like two split-KV partials and writes the result, and a
+//                 group starts a new unit only after that combination (its O is then free).
+// Tensor memory: NSB S buffers of 64 columns, then O of group 0 and O of group 1 (128 columns
+// each).  Every wait is bounded; on a timeout all roles stop, each MMA issuer waits (bounded) for
+// its own MMAs, all meet at the final barrier and warp 1 frees the tensor memory.
 #pragma once
 
 #include "attn_kernels.cuh"
@@ -35,13 +41,14 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
 template <int NSB>
 struct TcCols {
-    static constexpr uint32_t kO = NSB * 64;                     // O columns [kO, kO + 128)
-    static constexpr uint32_t kAlloc = (NSB * 64 + 128) <= 256 ? 256 : 512;
+    static constexpr uint32_t kO = NSB * 64;                     // O of group g: [kO + 128 g, + 128)
+    static constexpr uint32_t kAlloc = (NSB * 64 + 256) <= 256 ? 256 : 512;
+    static_assert(NSB * 64 + 256 <= 512, "tensor memory holds NSB S buffers and two O");
 };
 
 template <int NK, int NV, int NSB>
@@ -55,9 +62,11 @@ struct TcLayout {
     static constexpr int kPBytes = kHalfBytes;
     static constexpr int kBarOff = kPOff + NSB * kPBytes;
     // kfull[NK] kempty[NK] vfull[NV] vempty[NV] q_full[2] q_free[2] s_full[NSB] s_free[NSB]
-    // p_full[NSB] p_free[NSB] mma_done[2]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 * NSB + 2;
-    static constexpr int kKMetaOff = kBarOff + kNumBars * 8;
+    // p_full[NSB] p_free[NSB] mma_done[2] merge_done
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 * NSB + 3;
+    static constexpr int kPubOff = kBarOff + kNumBars * 8;        // per group: max[64], sum[64]
+    static constexpr int kPubUnitOff = kPubOff + 2 * 2 * 64 * 4;  // per group: its last tile's unit
+    static constexpr int kKMetaOff = kPubUnitOff + 16;
     static constexpr int kSMetaOff = kKMetaOff + NK * (int)sizeof(TileMeta);
     static constexpr int kPMetaOff = kSMetaOff + NSB * (int)sizeof(TileMeta);
     static constexpr int kPlanOff = kPMetaOff + NSB * (int)sizeof(TileMeta);
@@ -97,6 +106,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     uint64_t* p_full = s_free + NSB;
     uint64_t* p_free = p_full + NSB;
     uint64_t* mma_done = p_free + NSB;
+    uint64_t* merge_done = mma_done + 2;
+    float* pub = reinterpret_cast<float*>(smem + L::kPubOff);           // [group][max | sum][row]
+    volatile int* pub_unit = reinterpret_cast<volatile int*>(smem + L::kPubUnitOff);
     TileMeta* kmeta = reinterpret_cast<TileMeta*>(smem + L::kKMetaOff);
     TileMeta* smeta = reinterpret_cast<TileMeta*>(smem + L::kSMetaOff);
     TileMeta* pmeta = reinterpret_cast<TileMeta*>(smem + L::kPMetaOff);
@@ -142,6 +154,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             }
             mbar_init(&mma_done[0], 1);
             mbar_init(&mma_done[1], 1);
+            mbar_init(merge_done, 4);
+            pub_unit[0] = -1;
+            pub_unit[1] = -1;
             fence_barrier_init();
         }
     }
@@ -168,12 +183,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             TileWalker<SRC> walk;
             walk.init(a, plan_tiles);
             uint32_t uidx = 0, it = 0;
+            int ord = 0;
             const uint32_t q_bytes = (uint32_t)a.rows_total * 256u;
             bool alive = true;
             for (long long t = t_begin; t < t_end; ++t, ++it) {
                 TileMeta m;
                 int ty = 0, tz = 0;
                 walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
+                m.ord = ord;
+                if (m.flags & kLast) ++ord;
                 if (is_k) {
                     if (m.flags & kFirst) {
                         const uint32_t qb = uidx & 1u;
@@ -259,23 +277,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             constexpr uint32_t kIdescO = tc::idesc_bf16_f32(64, 128, false, true);
             const uint64_t dP = tc::smem_desc(smem_addr(smem + L::kPOff), 16, 1024);
             const uint64_t dV = tc::smem_desc(smem_addr(smem + L::kVOff), 8192, 1024);
-            uint32_t o_init = 0;
+            uint32_t o_init[2] = {0u, 0u};
+            int o_unit[2] = {-1, -1};
             for (uint32_t t = 0; t < n; ++t) {
-                const uint32_t sb = t % NSB, vs = t % NV;
-                // the softmax warps have written P(t) (and read this tile's description) by now
+                const uint32_t sb = t % NSB, vs = t % NV, g = t & 1u;
+                // the softmax group of tile t has written P(t) (and read its description) by now
                 if (!mbar_wait_bounded(&p_full[sb], (t / NSB) & 1u)) break;
                 const TileMeta m = pmeta[sb];
                 if (!mbar_wait_bounded(&vfull[vs], (t / NV) & 1u)) break;
                 tc::fence_after_sync();
-                if (m.flags & kFirst) o_init = 0;
+                if (m.unit != o_unit[g]) { o_unit[g] = m.unit; o_init[g] = 0u; }
                 if (m.nvalid > 0) {
                     const uint32_t poff = sb * (uint32_t)L::kPBytes;
                     const uint32_t voff = vs * (uint32_t)kTileBytes;
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        tc::mma_f16_ss(tmem + TCOL::kO, dP + ((poff + 32u * j) >> 4),
-                                       dV + ((voff + 2048u * j) >> 4), kIdescO, (o_init | (uint32_t)j) != 0u);
-                    o_init = 1;
+                        tc::mma_f16_ss(tmem + TCOL::kO + 128u * g, dP + ((poff + 32u * j) >> 4),
+                                       dV + ((voff + 2048u * j) >> 4), kIdescO, (o_init[g] | (uint32_t)j) != 0u);
+                    o_init[g] = 1u;
                 }
                 tc::commit(&p_free[sb]);
                 tc::commit(&vempty[vs]);
@@ -284,22 +303,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             mbar_wait_bounded(&mma_done[1], 0);
         }
     } else {
-        // =========================== softmax warps ===========================================
+        // =========================== softmax warps (two groups) ==============================
+        const uint32_t grp = warp >= 8 ? 1u : 0u;
+        const int gwarp0 = grp ? 8 : 2;                  // the group's first warp
+        const int gtid = threadIdx.x - 32 * gwarp0;      // 0 .. 127 within the group
         const int sp = warp & 3;
         const int half = lane >> 4;
         const int row = 16 * sp + (lane & 15);
         const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+        const uint32_t o_own = TCOL::kO + 128u * grp, o_oth = TCOL::kO + 128u * (grp ^ 1u);
+        float* pub_m_own = pub + (2 * grp) * 64;
+        float* pub_l_own = pub + (2 * grp + 1) * 64;
+        const float* pub_m_oth = pub + (2 * (grp ^ 1u)) * 64;
+        const float* pub_l_oth = pub + (2 * (grp ^ 1u) + 1) * 64;
         float m_used = -INFINITY, l_part = 0.f;
         unsigned long long vis = 0ull;
         bool row_ok = false;
-        int Lpre = 0;
+        int Lpre = 0, my_unit = -1;
         bool alive = true;
-        for (uint32_t it = 0; it < n && alive; ++it) {
+        for (uint32_t it = grp; it < n && alive; it += 2) {
             const uint32_t sb = it % NSB;
             if (!mbar_wait_bounded(&s_full[sb], (it / NSB) & 1u)) { alive = false; break; }
             tc::fence_after_sync();
             const TileMeta m = smeta[sb];
-            if (m.flags & kFirst) {
+            if (m.unit != my_unit) {
+                // first tile of a unit for this group: the previous unit's combination (which
+                // reads this group's O) must be done before this group's O is overwritten
+                if (m.ord >= 1 && !mbar_wait_bounded(merge_done, (uint32_t)(m.ord - 1) & 1u)) {
+                    alive = false;
+                    break;
+                }
+                my_unit = m.unit;
                 Lpre = m.L_tot - a.n_q;
                 const int R = m.rb * kRowsPerBlock + row;
                 row_ok = R < a.rows_total;
@@ -334,8 +368,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             }
             // ---- maximum over the row (both half-warps), running maximum -------------------
             float x[32];
+            if (mk == ~0u) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = ((mk >> j) & 1u) ? __uint_as_float(sr[j]) : -INFINITY;
+                for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sr[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) x[j] = ((mk >> j) & 1u) ? __uint_as_float(sr[j]) : -INFINITY;
+            }
             float mx8[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(fmaxf(x[j], x[j + 8]), fmaxf(x[j + 16], x[j + 24]));
@@ -383,57 +422,92 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 if (!mbar_wait_bounded(&vfull[vs], (it / NV) & 1u)) { alive = false; break; }
                 uint8_t* vt = smem + L::kVOff + vs * kTileBytes;
                 const int nrow = kTileKeys - m.nvalid;
-                for (int idx = threadIdx.x - 64; idx < nrow * 16; idx += 128) {
+                for (int idx = gtid; idx < nrow * 16; idx += 128) {
                     const int r = m.nvalid + idx / 16, c16 = idx % 16;
                     *reinterpret_cast<uint4*>(vt + (c16 >> 3) * kHalfBytes + r * 128 + (c16 & 7) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
             }
-            // ---- rare: move this warp's O rows to the new maximum (after PV of tile it - 1) --
+            // ---- rare: move this warp's O rows to the new maximum (after this group's
+            //      previous PV, tile it - 2, is done) --------------------------------------------
             if (__any_sync(0xffffffffu, rescale)) {
-                const uint32_t pb = (it - 1) % NSB;
-                if (!mbar_wait_bounded(&p_free[pb], ((it - 1) / NSB) & 1u)) { alive = false; break; }
+                if (it >= 2u) {
+                    const uint32_t pb = (it - 2u) % NSB;
+                    if (!mbar_wait_bounded(&p_free[pb], ((it - 2u) / NSB) & 1u)) { alive = false; break; }
+                }
                 tc::fence_after_sync();
                 const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[16];
                     __syncwarp();
-                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + TCOL::kO + 16u * c, o);
+                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + o_own + 16u * c, o);
                     tc::wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-                    tc::st_16x32bx2_x16<64>(tmem + lane_base + TCOL::kO + 16u * c, o);
+                    tc::st_16x32bx2_x16<64>(tmem + lane_base + o_own + 16u * c, o);
                 }
                 tc::wait_st();
             }
-            if (warp == 2 && lane == 0) pmeta[sb] = m;   // the PV issuer's copy of the description
+            // ---- publish this group's row state for the unit-end combination -----------------
+            const float l_row = l_part + __shfl_xor_sync(0xffffffffu, l_part, 16);
+            if (half == 0) {
+                pub_m_own[row] = m_used;
+                pub_l_own[row] = l_row;
+            }
+            if (warp == gwarp0 && lane == 0) {
+                pmeta[sb] = m;                           // the PV issuer's copy of the description
+                pub_unit[grp] = m.unit;
+            }
             fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[sb]);
-            // ---- unit end: O rows out of tensor memory ---------------------------------------
+            // ---- unit end: combine both groups' (O, max, sum), write the rows ----------------
             if (m.flags & kLast) {
                 if (!mbar_wait_bounded(&p_free[sb], (it / NSB) & 1u)) { alive = false; break; }
+                // the other group's last tile of this unit, if any, is tile it - 1: its P (and so
+                // its published state) is complete once its p_full phase has, and its PV before
+                // ours
+                bool other = false;
+                float m_o = -INFINITY, l_o = 0.f;
+                if (it >= 1u) {
+                    const uint32_t pb = (it - 1u) % NSB;
+                    if (!mbar_wait_bounded(&p_full[pb], ((it - 1u) / NSB) & 1u)) { alive = false; break; }
+                    if (pub_unit[grp ^ 1u] == m.unit) {
+                        other = true;
+                        m_o = pub_m_oth[row];
+                        l_o = pub_l_oth[row];
+                    }
+                }
                 tc::fence_after_sync();
-                const float l_sum = l_part + __shfl_xor_sync(0xffffffffu, l_part, 16);
+                const float M = fmaxf(m_used, m_o);
+                const float w_own = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
+                const float w_oth = (!other || m_o == -INFINITY) ? 0.f : fast_exp2(m_o - M);
+                const float l_sum = l_row * w_own + l_o * w_oth;
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                const float lse2 = l_sum > 0.f ? m_used + __log2f(l_sum) : -INFINITY;
+                const float lse2 = l_sum > 0.f ? M + __log2f(l_sum) : -INFINITY;
+                const bool use_own = w_own > 0.f, use_oth = w_oth > 0.f;
                 const int R = m.rb * kRowsPerBlock + row;
                 const int i = R / a.G, g = R - (R / a.G) * a.G;
                 const size_t orow = ((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g;
                 const int slot = (int)blockIdx.x + m.unit;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t o[16];
+                    uint32_t o[16], o2[16];
                     __syncwarp();
-                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + TCOL::kO + 16u * c, o);
+                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + o_own + 16u * c, o);
+                    tc::ld_16x32bx2_x16<64>(tmem + lane_base + o_oth + 16u * c, o2);
                     tc::wait_ld();
                     if (row_ok) {
                         const int d0 = 64 * half + 16 * c;
                         float v[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) v[j] = l_sum > 0.f ? __uint_as_float(o[j]) * inv : 0.f;
+                        for (int j = 0; j < 16; ++j) {
+                            float acc = use_own ? __uint_as_float(o[j]) * w_own : 0.f;
+                            if (use_oth) acc += __uint_as_float(o2[j]) * w_oth;
+                            v[j] = acc * inv;
+                        }
                         if (m.flags & kWhole) {
                             uint4* op = reinterpret_cast<uint4*>(a.out + orow * kD + d0);
                             op[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
@@ -458,6 +532,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                     }
                 }
                 tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(merge_done);
             }
         }
     }

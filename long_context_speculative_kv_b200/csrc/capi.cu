@@ -255,7 +255,7 @@ bool use_tc(const Shape& s) {
 char tc_variant() {
     static char v = [] {
         const char* e = std::getenv("WMTP_TC_VARIANT");
-        return (e && e[0] == 'B') ? 'B' : 'A';
+        return (e && (e[0] == 'B' || e[0] == 'C' || e[0] == 'D')) ? e[0] : 'A';
     }();
     return v;
 }
@@ -289,6 +289,8 @@ int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, 
                    int sm_count, const Shape& s, cudaStream_t st) {
     switch (tc_variant()) {
         case 'B': return launch_attn_tc_t<SRC, 4, 3, 2>(km, vm, q, a, sm_count, s, st);
+        case 'C': return launch_attn_tc_t<SRC, 4, 6, 3>(km, vm, q, a, sm_count, s, st);
+        case 'D': return launch_attn_tc_t<SRC, 5, 5, 3>(km, vm, q, a, sm_count, s, st);
         default: return launch_attn_tc_t<SRC, 6, 4, 3>(km, vm, q, a, sm_count, s, st);
     }
 }
