@@ -140,25 +140,49 @@ template <int SRC>
 struct TileWalker {
     int b = 0;
     long long b_start = 0, per_b = 0;
+    // position of the last described tile, for the O(1) step to the next one (producers walk
+    // their ranges in order; a division-free step keeps the producer loop short)
+    long long cur_t = -1;
+    int nt_b = 0, unit_in_b = 0, tile = 0;
+    // page id of the next tile, loaded one step ahead so its latency hides behind this step
+    int pf_b = -1, pf_tile = -1, pf_page = -1;
 
     __device__ __forceinline__ void init(const AttnArgs& a, const int* plan_tiles) {
         b = 0;
         b_start = 0;
         per_b = (long long)plan_tiles[0] * a.Hkv * a.n_rb;
+        cur_t = -1;
     }
 
     __device__ __forceinline__ void describe(const AttnArgs& a, const int* plan_tiles,
                                              const int* plan_len, long long t, long long t_begin,
                                              long long t_end, TileMeta& m, int& ty, int& tz) {
-        while (t >= b_start + per_b) {
-            b_start += per_b;
-            ++b;
-            per_b = (long long)plan_tiles[b] * a.Hkv * a.n_rb;
+        const int units_b = a.Hkv * a.n_rb;
+        if (cur_t >= 0 && t == cur_t + 1) {
+            if (++tile == nt_b) {
+                tile = 0;
+                if (++unit_in_b == units_b) {
+                    unit_in_b = 0;
+                    b_start += per_b;
+                    do {
+                        ++b;
+                        per_b = (long long)plan_tiles[b] * units_b;
+                    } while (per_b == 0);              // t < total tiles: some later request has tiles
+                    nt_b = plan_tiles[b];
+                }
+            }
+        } else {
+            while (t >= b_start + per_b) {
+                b_start += per_b;
+                ++b;
+                per_b = (long long)plan_tiles[b] * units_b;
+            }
+            nt_b = plan_tiles[b];
+            const long long off = t - b_start;
+            unit_in_b = (int)(off / nt_b);
+            tile = (int)(off - (long long)unit_in_b * nt_b);
         }
-        const int nt_b = plan_tiles[b];
-        const long long off = t - b_start;
-        const int unit_in_b = (int)(off / nt_b);
-        const int tile = (int)(off - (long long)unit_in_b * nt_b);
+        cur_t = t;
         const int h = unit_in_b / a.n_rb;
         const int rb = unit_in_b - h * a.n_rb;
         const long long u_start = b_start + (long long)unit_in_b * nt_b;
@@ -169,7 +193,18 @@ struct TileWalker {
                   ((t == t_end - 1 || tile == nt_b - 1) ? kLast : 0) |
                   ((u_start >= t_begin && u_start + nt_b <= t_end) ? kWhole : 0);
         if (SRC == kSrcPaged) {
-            const int page = tile < a.max_pages ? a.page_table[(size_t)b * a.max_pages + tile] : -1;
+            int page;
+            if (pf_b == b && pf_tile == tile) {
+                page = pf_page;
+            } else {
+                page = tile < a.max_pages ? a.page_table[(size_t)b * a.max_pages + tile] : -1;
+            }
+            // next tile of this request: the following tile of this unit, or tile 0 of the next
+            // unit (the same pages, another kv head or row block)
+            const int nxt = (tile + 1 < nt_b) ? tile + 1 : 0;
+            pf_b = b;
+            pf_tile = nxt;
+            pf_page = nxt < a.max_pages ? a.page_table[(size_t)b * a.max_pages + nxt] : -1;
             m.pos0 = tile * kTileKeys;
             const int rem = m.L_tot - m.pos0;
             m.nvalid = rem < kTileKeys ? rem : kTileKeys;

@@ -44,32 +44,41 @@ namespace wmtp {
 constexpr int kTcThreads = 384;
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
+// Tiles go in pairs (CTA-local tiles 2q and 2q + 1): pair q's K tiles share one K slot and one
+// S buffer of 128 columns, so a pair of the same unit needs one N = 128 QK^T instead of two
+// N = 64 ones (the tensor core's cost per tile drops from ~656 to ~512 cycles).
+constexpr int kTcPBufs = 4;                  // P buffers (one tile each)
+
 template <int NSB>
 struct TcCols {
-    static constexpr uint32_t kO = NSB * 64;                     // O of group g: [kO + 128 g, + 128)
-    static constexpr uint32_t kAlloc = (NSB * 64 + 256) <= 256 ? 256 : 512;
-    static_assert(NSB * 64 + 256 <= 512, "tensor memory holds NSB S buffers and two O");
+    static constexpr uint32_t kO = NSB * 128;                    // O of group g: [kO + 128 g, + 128)
+    static constexpr uint32_t kAlloc = 512;
+    static_assert(NSB * 128 + 256 <= 512, "tensor memory holds NSB S pair buffers and two O");
 };
 
+// K ring: NK pair slots of 32 KiB laid out [tile 0, dims 0-63][tile 1, dims 0-63][tile 0, dims
+// 64-127][tile 1, dims 64-127], so 128 keys of one 64-dim half are 128 consecutive 128-byte rows
+// (the K-major operand of an N = 128 MMA).
 template <int NK, int NV, int NSB>
 struct TcLayout {
     static constexpr int kTileHalf = kHalfBytes;                 // 64 rows x 128 bytes
-    static constexpr int kKOff = 0;                              // NK x [64 keys][128] (2 boxes)
-    static constexpr int kVOff = kKOff + NK * kTileBytes;        // NV x [64 keys][128]
+    static constexpr int kKSlotBytes = 2 * kTileBytes;
+    static constexpr int kKOff = 0;                              // NK x pair slot
+    static constexpr int kVOff = kKOff + NK * kKSlotBytes;       // NV x [64 keys][128]
     static constexpr int kQOff = kVOff + NV * kTileBytes;        // 2 x [64 rows][128]
     static constexpr int kQBytes = kTileBytes;
-    static constexpr int kPOff = kQOff + 2 * kQBytes;            // NSB x [64 rows][64 keys]
+    static constexpr int kPOff = kQOff + 2 * kQBytes;            // kTcPBufs x [64 rows][64 keys]
     static constexpr int kPBytes = kHalfBytes;
-    static constexpr int kBarOff = kPOff + NSB * kPBytes;
+    static constexpr int kBarOff = kPOff + kTcPBufs * kPBytes;
     // kfull[NK] kempty[NK] vfull[NV] vempty[NV] q_full[2] q_free[2] s_full[NSB] s_free[NSB]
-    // p_full[NSB] p_free[NSB] mma_done[2] merge_done
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 * NSB + 3;
+    // p_full[P] p_free[P] mma_done[2] merge_done
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 2 * NSB + 2 * kTcPBufs + 3;
     static constexpr int kPubOff = kBarOff + kNumBars * 8;        // per group: max[64], sum[64]
     static constexpr int kPubUnitOff = kPubOff + 2 * 2 * 64 * 4;  // per group: its last tile's unit
     static constexpr int kKMetaOff = kPubUnitOff + 16;
-    static constexpr int kSMetaOff = kKMetaOff + NK * (int)sizeof(TileMeta);
-    static constexpr int kPMetaOff = kSMetaOff + NSB * (int)sizeof(TileMeta);
-    static constexpr int kPlanOff = kPMetaOff + NSB * (int)sizeof(TileMeta);
+    static constexpr int kSMetaOff = kKMetaOff + 2 * NK * (int)sizeof(TileMeta);
+    static constexpr int kPMetaOff = kSMetaOff + 2 * NSB * (int)sizeof(TileMeta);
+    static constexpr int kPlanOff = kPMetaOff + kTcPBufs * (int)sizeof(TileMeta);
     static constexpr int kPlanBytes = 2 * kMaxBatch * 4;
     static constexpr int kTmemOff = kPlanOff + kPlanBytes;
     static constexpr int kTotal = kTmemOff + 16;
@@ -104,8 +113,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     uint64_t* s_full = q_free + 2;
     uint64_t* s_free = s_full + NSB;
     uint64_t* p_full = s_free + NSB;
-    uint64_t* p_free = p_full + NSB;
-    uint64_t* mma_done = p_free + NSB;
+    uint64_t* p_free = p_full + kTcPBufs;
+    uint64_t* mma_done = p_free + kTcPBufs;
     uint64_t* merge_done = mma_done + 2;
     float* pub = reinterpret_cast<float*>(smem + L::kPubOff);           // [group][max | sum][row]
     volatile int* pub_unit = reinterpret_cast<volatile int*>(smem + L::kPubUnitOff);
@@ -143,12 +152,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             const long long c = blockIdx.x;
             s_range[0] = c < peff ? cta_begin(c, T, peff) : 0;
             s_range[1] = c < peff ? cta_begin(c + 1, T, peff) : 0;
-            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], 1); mbar_init(&kempty[k], 1); }
+            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], 2); mbar_init(&kempty[k], 1); }
             for (int k = 0; k < NV; ++k) { mbar_init(&vfull[k], 1); mbar_init(&vempty[k], 1); }
             for (int k = 0; k < 2; ++k) { mbar_init(&q_full[k], 1); mbar_init(&q_free[k], 1); }
             for (int k = 0; k < NSB; ++k) {
-                mbar_init(&s_full[k], 2);      // tensor-core completion + the forwarded description
-                mbar_init(&s_free[k], 4);
+                mbar_init(&s_full[k], 2);      // tensor-core completion + the forwarded descriptions
+                mbar_init(&s_free[k], 8);      // both groups' warps have read their tile's scores
+            }
+            for (int k = 0; k < kTcPBufs; ++k) {
                 mbar_init(&p_full[k], 4);
                 mbar_init(&p_free[k], 1);
             }
@@ -202,17 +213,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                         tma_load_4d(qdst + kHalfBytes, &qmap, &q_full[qb], 64, 0, m.h, m.b * a.n_q);
                         ++uidx;
                     }
-                    const uint32_t ks = it % NK;
-                    if (!mbar_wait_bounded(&kempty[ks], ((it / NK) & 1u) ^ 1u)) { alive = false; break; }
-                    kmeta[ks] = m;
-                    uint8_t* dst = smem + L::kKOff + ks * kTileBytes;
+                    const uint32_t pq = it >> 1, sub = it & 1u, ks = pq % NK;
+                    if (sub == 0u && !mbar_wait_bounded(&kempty[ks], ((pq / NK) & 1u) ^ 1u)) { alive = false; break; }
+                    kmeta[2 * ks + sub] = m;
+                    uint8_t* dst = smem + L::kKOff + ks * L::kKSlotBytes + sub * kHalfBytes;
                     if (m.nvalid > 0) {
                         mbar_arrive_expect_tx(&kfull[ks], kTileBytes);
                         tma_load_3d(dst, &kmap, &kfull[ks], 0, ty, tz, pol);
-                        tma_load_3d(dst + kHalfBytes, &kmap, &kfull[ks], 64, ty, tz, pol);
+                        tma_load_3d(dst + kTileBytes, &kmap, &kfull[ks], 64, ty, tz, pol);
                     } else {
                         mbar_arrive(&kfull[ks]);
                     }
+                    if (sub == 0u && t + 1 == t_end) mbar_arrive(&kfull[ks]);   // pair without tile 1
                 } else {
                     const uint32_t vs = it % NV;
                     if (!mbar_wait_bounded(&vempty[vs], ((it / NV) & 1u) ^ 1u)) { alive = false; break; }
@@ -228,44 +240,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             }
             // drain: every issued stage released (no copy still landing at exit)
             const uint32_t depth = is_k ? NK : NV;
+            const uint32_t used = is_k ? (it + 1) / 2 : it;          // K: pair slots
             uint64_t* empty = is_k ? kempty : vempty;
-            for (uint32_t k = (it > depth ? it - depth : 0); k < it && alive; ++k)
+            for (uint32_t k = (used > depth ? used - depth : 0); k < used && alive; ++k)
                 if (!mbar_wait_bounded(&empty[k % depth], (k / depth) & 1u)) break;
         }
     } else if (warp == 1) {
         // =========================== S issuer (QK^T) =========================================
         if (lane == 0) {
-            constexpr uint32_t kIdescS = tc::idesc_bf16_f32(64, 64, false, false);
+            constexpr uint32_t kIdescS64 = tc::idesc_bf16_f32(64, 64, false, false);
+            constexpr uint32_t kIdescS128 = tc::idesc_bf16_f32(64, 128, false, false);
             // descriptors of the ring bases; a k-step or buffer offset is added as (bytes >> 4)
             const uint64_t dK = tc::smem_desc(smem_addr(smem + L::kKOff), 16, 1024);
             const uint64_t dQ = tc::smem_desc(smem_addr(smem + L::kQOff), 16, 1024);
             uint32_t uidx = 0;
-            for (uint32_t t = 0; t < n; ++t) {
-                const uint32_t ks = t % NK;
-                if (!mbar_wait_bounded(&kfull[ks], (t / NK) & 1u)) break;
-                const TileMeta m = kmeta[ks];
-                if (m.flags & kFirst) {
-                    if (!mbar_wait_bounded(&q_full[uidx & 1u], (uidx >> 1) & 1u)) break;
-                    ++uidx;
+            const uint32_t npairs = (n + 1) / 2;
+            bool ok = true;
+            for (uint32_t pq = 0; pq < npairs && ok; ++pq) {
+                const uint32_t ks = pq % NK, sb = pq % NSB;
+                if (!mbar_wait_bounded(&kfull[ks], (pq / NK) & 1u)) break;
+                const bool has1 = 2 * pq + 1 < n;
+                TileMeta mt[2];
+                uint32_t qb[2] = {0u, 0u};
+                for (uint32_t sub = 0; sub < (has1 ? 2u : 1u); ++sub) {
+                    mt[sub] = kmeta[2 * ks + sub];
+                    if (mt[sub].flags & kFirst) {
+                        if (!mbar_wait_bounded(&q_full[uidx & 1u], (uidx >> 1) & 1u)) { ok = false; break; }
+                        ++uidx;
+                    }
+                    qb[sub] = (uidx - 1u) & 1u;
                 }
-                const uint32_t sb = t % NSB;
-                if (!mbar_wait_bounded(&s_free[sb], ((t / NSB) & 1u) ^ 1u)) break;
-                smeta[sb] = m;
+                if (!ok) break;
+                if (!mbar_wait_bounded(&s_free[sb], ((pq / NSB) & 1u) ^ 1u)) break;
+                smeta[2 * sb] = mt[0];
+                if (has1) smeta[2 * sb + 1] = mt[1];
                 tc::fence_after_sync();
-                if (m.nvalid > 0) {
-                    const uint32_t qoff = ((uidx - 1u) & 1u) * (uint32_t)L::kQBytes;
-                    const uint32_t koff = ks * (uint32_t)kTileBytes;
+                const uint32_t kslot = ks * (uint32_t)L::kKSlotBytes;
+                const bool paired = has1 && mt[0].nvalid > 0 && mt[1].nvalid > 0 && mt[0].unit == mt[1].unit;
+                if (paired) {
+                    // one N = 128 MMA per k-step: keys of both tiles are consecutive rows
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const uint32_t off = (uint32_t)((j >> 2) * kHalfBytes + (j & 3) * 32);
-                        tc::mma_f16_ss(tmem + sb * 64u, dQ + ((qoff + off) >> 4), dK + ((koff + off) >> 4),
-                                       kIdescS, j > 0);
+                        const uint32_t qoff = qb[0] * (uint32_t)L::kQBytes + (uint32_t)((j >> 2) * kHalfBytes + (j & 3) * 32);
+                        const uint32_t koff = kslot + (uint32_t)((j >> 2) * kTileBytes + (j & 3) * 32);
+                        tc::mma_f16_ss(tmem + sb * 128u, dQ + (qoff >> 4), dK + (koff >> 4), kIdescS128, j > 0);
+                    }
+                } else {
+                    for (uint32_t sub = 0; sub < (has1 ? 2u : 1u); ++sub) {
+                        if (mt[sub].nvalid <= 0) continue;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t qoff = qb[sub] * (uint32_t)L::kQBytes +
+                                                  (uint32_t)((j >> 2) * kHalfBytes + (j & 3) * 32);
+                            const uint32_t koff = kslot + sub * (uint32_t)kHalfBytes +
+                                                  (uint32_t)((j >> 2) * kTileBytes + (j & 3) * 32);
+                            tc::mma_f16_ss(tmem + sb * 128u + 64u * sub, dQ + (qoff >> 4), dK + (koff >> 4),
+                                           kIdescS64, j > 0);
+                        }
                     }
                 }
                 tc::commit(&kempty[ks]);
                 tc::commit(&s_full[sb]);
                 mbar_arrive(&s_full[sb]);
-                if (m.flags & kLast) tc::commit(&q_free[(uidx - 1u) & 1u]);
+                if (mt[0].flags & kLast) tc::commit(&q_free[qb[0]]);
+                if (has1 && (mt[1].flags & kLast)) tc::commit(&q_free[qb[1]]);
             }
             // every MMA of this thread complete before the tensor memory is freed
             tc::commit(&mma_done[0]);
@@ -280,9 +318,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             uint32_t o_init[2] = {0u, 0u};
             int o_unit[2] = {-1, -1};
             for (uint32_t t = 0; t < n; ++t) {
-                const uint32_t sb = t % NSB, vs = t % NV, g = t & 1u;
+                const uint32_t sb = t % kTcPBufs, vs = t % NV, g = t & 1u;
                 // the softmax group of tile t has written P(t) (and read its description) by now
-                if (!mbar_wait_bounded(&p_full[sb], (t / NSB) & 1u)) break;
+                if (!mbar_wait_bounded(&p_full[sb], (t / kTcPBufs) & 1u)) break;
                 const TileMeta m = pmeta[sb];
                 if (!mbar_wait_bounded(&vfull[vs], (t / NV) & 1u)) break;
                 tc::fence_after_sync();
@@ -322,10 +360,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         int Lpre = 0, my_unit = -1;
         bool alive = true;
         for (uint32_t it = grp; it < n && alive; it += 2) {
-            const uint32_t sb = it % NSB;
-            if (!mbar_wait_bounded(&s_full[sb], (it / NSB) & 1u)) { alive = false; break; }
+            const uint32_t sq = (it >> 1) % NSB;             // S pair buffer
+            const uint32_t scol = sq * 128u + 64u * grp;     // this tile's 64 score columns
+            const uint32_t sb = it % kTcPBufs;               // P buffer
+            if (!mbar_wait_bounded(&s_full[sq], ((it >> 1) / NSB) & 1u)) { alive = false; break; }
             tc::fence_after_sync();
-            const TileMeta m = smeta[sb];
+            const TileMeta m = smeta[2 * sq + grp];
             if (m.unit != my_unit) {
                 // first tile of a unit for this group: the previous unit's combination (which
                 // reads this group's O) must be done before this group's O is overwritten
@@ -344,12 +384,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             // ---- this thread's 32 scores from tensor memory ---------------------------------
             __syncwarp();
             uint32_t sr[32];
-            tc::ld_16x32bx2_x16<32>(tmem + lane_base + sb * 64u, sr);
-            tc::ld_16x32bx2_x16<32>(tmem + lane_base + sb * 64u + 16u, sr + 16);
+            tc::ld_16x32bx2_x16<32>(tmem + lane_base + scol, sr);
+            tc::ld_16x32bx2_x16<32>(tmem + lane_base + scol + 16u, sr + 16);
             tc::wait_ld();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sb]);
+            if (lane == 0) mbar_arrive(&s_free[sq]);
             // ---- key mask of this row: valid rows of the tile, prefix keys, visible step keys --
             uint32_t mk = 0u;
             if (row_ok && m.nvalid > 0) {
@@ -403,7 +443,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             }
             l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             // ---- P to shared memory (its buffer is free once PV of tile it - NSB is done) -----
-            if (it >= (uint32_t)NSB && !mbar_wait_bounded(&p_free[sb], ((it / NSB) & 1u) ^ 1u)) {
+            if (it >= (uint32_t)kTcPBufs && !mbar_wait_bounded(&p_free[sb], ((it / kTcPBufs) & 1u) ^ 1u)) {
                 alive = false;
                 break;
             }
@@ -432,8 +472,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             //      previous PV, tile it - 2, is done) --------------------------------------------
             if (__any_sync(0xffffffffu, rescale)) {
                 if (it >= 2u) {
-                    const uint32_t pb = (it - 2u) % NSB;
-                    if (!mbar_wait_bounded(&p_free[pb], ((it - 2u) / NSB) & 1u)) { alive = false; break; }
+                    const uint32_t pb = (it - 2u) % kTcPBufs;
+                    if (!mbar_wait_bounded(&p_free[pb], ((it - 2u) / kTcPBufs) & 1u)) { alive = false; break; }
                 }
                 tc::fence_after_sync();
                 const float f = rescale ? alpha : 1.f;
@@ -465,15 +505,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             if (lane == 0) mbar_arrive(&p_full[sb]);
             // ---- unit end: combine both groups' (O, max, sum), write the rows ----------------
             if (m.flags & kLast) {
-                if (!mbar_wait_bounded(&p_free[sb], (it / NSB) & 1u)) { alive = false; break; }
+                if (!mbar_wait_bounded(&p_free[sb], (it / kTcPBufs) & 1u)) { alive = false; break; }
                 // the other group's last tile of this unit, if any, is tile it - 1: its P (and so
                 // its published state) is complete once its p_full phase has, and its PV before
                 // ours
                 bool other = false;
                 float m_o = -INFINITY, l_o = 0.f;
                 if (it >= 1u) {
-                    const uint32_t pb = (it - 1u) % NSB;
-                    if (!mbar_wait_bounded(&p_full[pb], ((it - 1u) / NSB) & 1u)) { alive = false; break; }
+                    const uint32_t pb = (it - 1u) % kTcPBufs;
+                    if (!mbar_wait_bounded(&p_full[pb], ((it - 1u) / kTcPBufs) & 1u)) { alive = false; break; }
                     if (pub_unit[grp ^ 1u] == m.unit) {
                         other = true;
                         m_o = pub_m_oth[row];

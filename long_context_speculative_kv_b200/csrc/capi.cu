@@ -250,12 +250,12 @@ bool use_tc(const Shape& s) {
     return mode == 2 || (mode == 1 && s.rows_blk > 32);
 }
 
-// tcgen05 kernel variants (K ring, V ring, S/P buffers), one CTA per SM: A = (6, 4, 3),
-// B = (4, 3, 2).  WMTP_TC_VARIANT=B selects B (sweeps).
+// tcgen05 kernel variants (K pair slots, V ring, S pair buffers), one CTA per SM: A = (3, 3, 2),
+// B = (2, 4, 2), C = (2, 5, 2).  WMTP_TC_VARIANT=B|C selects another (sweeps).
 char tc_variant() {
     static char v = [] {
         const char* e = std::getenv("WMTP_TC_VARIANT");
-        return (e && (e[0] == 'B' || e[0] == 'C' || e[0] == 'D')) ? e[0] : 'A';
+        return (e && (e[0] == 'B' || e[0] == 'C')) ? e[0] : 'A';
     }();
     return v;
 }
@@ -288,10 +288,9 @@ template <int SRC>
 int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
                    int sm_count, const Shape& s, cudaStream_t st) {
     switch (tc_variant()) {
-        case 'B': return launch_attn_tc_t<SRC, 4, 3, 2>(km, vm, q, a, sm_count, s, st);
-        case 'C': return launch_attn_tc_t<SRC, 4, 6, 3>(km, vm, q, a, sm_count, s, st);
-        case 'D': return launch_attn_tc_t<SRC, 5, 5, 3>(km, vm, q, a, sm_count, s, st);
-        default: return launch_attn_tc_t<SRC, 6, 4, 3>(km, vm, q, a, sm_count, s, st);
+        case 'B': return launch_attn_tc_t<SRC, 2, 4, 2>(km, vm, q, a, sm_count, s, st);
+        case 'C': return launch_attn_tc_t<SRC, 2, 5, 2>(km, vm, q, a, sm_count, s, st);
+        default: return launch_attn_tc_t<SRC, 3, 3, 2>(km, vm, q, a, sm_count, s, st);
     }
 }
 
