@@ -297,7 +297,9 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     static_assert(KPW % 16 == 0, "keys per warp must be a multiple of 16");
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base for the 128-byte swizzle, by pointer arithmetic on the shared array
+    // (an integer round trip would make every access through it a generic one)
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     float* merge_o = reinterpret_cast<float*>(smem + L::kMergeOff);
     float* merge_ml = reinterpret_cast<float*>(smem + L::kMergeMLOff);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff);

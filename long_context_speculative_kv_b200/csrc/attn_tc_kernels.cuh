@@ -41,13 +41,14 @@
 
 namespace wmtp {
 
-constexpr int kTcThreads = 384;
+// 384 threads; with fp8 KV four more warps (12..15) widen the fp8 tiles into fp16 operands.
+template <bool KV8>
+constexpr int tc_threads() { return KV8 ? 512 : 384; }
 constexpr float kRescaleThreshold = 8.f;   // log2 units
 
 // Tiles go in pairs (CTA-local tiles 2q and 2q + 1): pair q's K tiles share one K slot and one
 // S buffer of 128 columns, so a pair of the same unit needs one N = 128 QK^T instead of two
 // N = 64 ones (the tensor core's cost per tile drops from ~656 to ~512 cycles).
-constexpr int kTcPBufs = 4;                  // P buffers (one tile each)
 
 template <int NSB>
 struct TcCols {
@@ -59,26 +60,32 @@ struct TcCols {
 // K ring: NK pair slots of 32 KiB laid out [tile 0, dims 0-63][tile 1, dims 0-63][tile 0, dims
 // 64-127][tile 1, dims 64-127], so 128 keys of one 64-dim half are 128 consecutive 128-byte rows
 // (the K-major operand of an N = 128 MMA).
-template <int NK, int NV, int NSB>
+// fp8 KV: the producers land each E4M3 tile (one 128-byte x 64-key box) in the upper 64-dim half
+// of its fp16 slot, and the converter warps widen it in place (see widen_rows).
+template <int NK, int NV, int NSB, bool KV8 = false>
 struct TcLayout {
+    static constexpr int kPBufs = 4;                             // P buffers (one tile each)
+    static constexpr int kStage8 = KV8 ? 1 : 0;                  // (fp8: per-slot landing barriers)
     static constexpr int kTileHalf = kHalfBytes;                 // 64 rows x 128 bytes
     static constexpr int kKSlotBytes = 2 * kTileBytes;
     static constexpr int kKOff = 0;                              // NK x pair slot
     static constexpr int kVOff = kKOff + NK * kKSlotBytes;       // NV x [64 keys][128]
     static constexpr int kQOff = kVOff + NV * kTileBytes;        // 2 x [64 rows][128]
     static constexpr int kQBytes = kTileBytes;
-    static constexpr int kPOff = kQOff + 2 * kQBytes;            // kTcPBufs x [64 rows][64 keys]
+    static constexpr int kPOff = kQOff + 2 * kQBytes;            // kPBufs x [64 rows][64 keys]
     static constexpr int kPBytes = kHalfBytes;
-    static constexpr int kBarOff = kPOff + kTcPBufs * kPBytes;
+    static constexpr int kBarOff = kPOff + kPBufs * kPBytes;
     // kfull[NK] kempty[NK] vfull[NV] vempty[NV] q_full[2] q_free[2] s_full[NSB] s_free[NSB]
-    // p_full[P] p_free[P] mma_done[2] merge_done
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 2 * NSB + 2 * kTcPBufs + 3;
+    // p_full[P] p_free[P] mma_done[2] merge_done; fp8: k8full[2 NK] v8full[NV] (codes landed),
+    // q_conv[2]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 2 * NSB + 2 * kPBufs + 3 +
+                                    kStage8 * (2 * NK + NV) + 2;
     static constexpr int kPubOff = kBarOff + kNumBars * 8;        // per group: max[64], sum[64]
     static constexpr int kPubUnitOff = kPubOff + 2 * 2 * 64 * 4;  // per group: its last tile's unit
     static constexpr int kKMetaOff = kPubUnitOff + 16;
     static constexpr int kSMetaOff = kKMetaOff + 2 * NK * (int)sizeof(TileMeta);
     static constexpr int kPMetaOff = kSMetaOff + 2 * NSB * (int)sizeof(TileMeta);
-    static constexpr int kPlanOff = kPMetaOff + kTcPBufs * (int)sizeof(TileMeta);
+    static constexpr int kPlanOff = kPMetaOff + kPBufs * (int)sizeof(TileMeta);
     static constexpr int kPlanBytes = 2 * kMaxBatch * 4;
     static constexpr int kTmemOff = kPlanOff + kPlanBytes;
     static constexpr int kTotal = kTmemOff + 16;
@@ -95,14 +102,56 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-template <int SRC, int NK, int NV, int NSB>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// Widens one fp8 tile in place.  The E4M3 codes (a 128-byte x 64-key TMA box, 128-byte swizzle)
+// sit where the fp16 tile's upper half (dims 64-127) goes; `lo` is the fp16 lower half.  Thread
+// r (0 .. 63) owns key row r: it reads its whole code row, then writes dims 0-63 into `lo` and
+// dims 64-127 over the code row it has just read (no other row is touched, so no thread can
+// overwrite codes another still needs).  Rows at or past `nvalid` become zeros.
+__device__ __forceinline__ void widen_rows(uint32_t codes_hi, uint32_t lo, int nvalid, int r) {
+    uint32_t w[32];
+    if (r < nvalid) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[4 * c]), "=r"(w[4 * c + 1]), "=r"(w[4 * c + 2]), "=r"(w[4 * c + 3])
+                         : "r"(codes_hi + (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4))));
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        // codes 16 c .. 16 c + 15 -> fp16 dims 16 c .. 16 c + 15: half c / 4, chunks 2 (c % 4), + 1
+        uint32_t h[8];
+        if (r < nvalid) {
+            e4m3x4_to_f16x2x2(w[4 * c], h[0], h[1]);
+            e4m3x4_to_f16x2x2(w[4 * c + 1], h[2], h[3]);
+            e4m3x4_to_f16x2x2(w[4 * c + 2], h[4], h[5]);
+            e4m3x4_to_f16x2x2(w[4 * c + 3], h[6], h[7]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = 0u;
+        }
+        const uint32_t hb = ((c >> 2) ? codes_hi : lo) + (uint32_t)(r * 128);
+        const int c0 = 2 * (c & 3);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                     :: "r"(hb + (uint32_t)((c0 ^ (r & 7)) << 4)), "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3])
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                     :: "r"(hb + (uint32_t)(((c0 + 1) ^ (r & 7)) << 4)), "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
+                     : "memory");
+    }
+}
+
+template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
+__global__ void __launch_bounds__(tc_threads<KV8>(), 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                const __grid_constant__ CUtensorMap qmap, const AttnArgs a) {
-    using L = TcLayout<NK, NV, NSB>;
+    using L = TcLayout<NK, NV, NSB, KV8>;
+    constexpr int kPB = L::kPBufs;
+    constexpr int kS8 = L::kStage8;
     using TCOL = TcCols<NSB>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base for the 128-byte swizzle, by pointer arithmetic on the shared array
+    // (an integer round trip would make every access through it a generic one)
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
     uint64_t* kfull = bars;
     uint64_t* kempty = kfull + NK;
@@ -113,9 +162,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     uint64_t* s_full = q_free + 2;
     uint64_t* s_free = s_full + NSB;
     uint64_t* p_full = s_free + NSB;
-    uint64_t* p_free = p_full + kTcPBufs;
-    uint64_t* mma_done = p_free + kTcPBufs;
+    uint64_t* p_free = p_full + kPB;
+    uint64_t* mma_done = p_free + kPB;
     uint64_t* merge_done = mma_done + 2;
+    uint64_t* k8full = merge_done + 1;                  // fp8: [2 NK] codes of tile (slot, sub) landed
+    uint64_t* v8full = k8full + kS8 * 2 * NK;           // fp8: [NV]
+    uint64_t* q_conv = v8full + kS8 * NV;
     float* pub = reinterpret_cast<float*>(smem + L::kPubOff);           // [group][max | sum][row]
     volatile int* pub_unit = reinterpret_cast<volatile int*>(smem + L::kPubUnitOff);
     TileMeta* kmeta = reinterpret_cast<TileMeta*>(smem + L::kKMetaOff);
@@ -152,14 +204,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             const long long c = blockIdx.x;
             s_range[0] = c < peff ? cta_begin(c, T, peff) : 0;
             s_range[1] = c < peff ? cta_begin(c + 1, T, peff) : 0;
-            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], 2); mbar_init(&kempty[k], 1); }
-            for (int k = 0; k < NV; ++k) { mbar_init(&vfull[k], 1); mbar_init(&vempty[k], 1); }
+            // K pair slot: one arrival per tile (bf16: the producer; fp8: each converter warp)
+            // (fp8: two converter warps for K and two for V, one arrival each per tile)
+            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], KV8 ? 4 : 2); mbar_init(&kempty[k], 1); }
+            for (int k = 0; k < NV; ++k) { mbar_init(&vfull[k], KV8 ? 2 : 1); mbar_init(&vempty[k], 1); }
+            if (KV8) {
+                for (int k = 0; k < 2 * NK; ++k) mbar_init(&k8full[k], 1);
+                for (int k = 0; k < NV; ++k) mbar_init(&v8full[k], 1);
+                mbar_init(&q_conv[0], 2);
+                mbar_init(&q_conv[1], 2);
+            }
             for (int k = 0; k < 2; ++k) { mbar_init(&q_full[k], 1); mbar_init(&q_free[k], 1); }
             for (int k = 0; k < NSB; ++k) {
                 mbar_init(&s_full[k], 2);      // tensor-core completion + the forwarded descriptions
                 mbar_init(&s_free[k], 8);      // both groups' warps have read their tile's scores
             }
-            for (int k = 0; k < kTcPBufs; ++k) {
+            for (int k = 0; k < kPB; ++k) {
                 mbar_init(&p_full[k], 4);
                 mbar_init(&p_free[k], 1);
             }
@@ -216,6 +276,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                     const uint32_t pq = it >> 1, sub = it & 1u, ks = pq % NK;
                     if (sub == 0u && !mbar_wait_bounded(&kempty[ks], ((pq / NK) & 1u) ^ 1u)) { alive = false; break; }
                     kmeta[2 * ks + sub] = m;
+                    if (KV8) {
+                        // fp8: the codes land in the tile's upper half; the converters widen them
+                        uint64_t* lb = &k8full[2 * ks + sub];
+                        if (m.nvalid > 0) {
+                            mbar_arrive_expect_tx(lb, kTileBytes8);
+                            tma_load_3d(smem + L::kKOff + ks * L::kKSlotBytes + kTileBytes + sub * kHalfBytes,
+                                        &kmap, lb, 0, ty, tz, pol);
+                        } else {
+                            mbar_arrive(lb);
+                        }
+                        continue;
+                    }
                     uint8_t* dst = smem + L::kKOff + ks * L::kKSlotBytes + sub * kHalfBytes;
                     if (m.nvalid > 0) {
                         mbar_arrive_expect_tx(&kfull[ks], kTileBytes);
@@ -225,6 +297,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                         mbar_arrive(&kfull[ks]);
                     }
                     if (sub == 0u && t + 1 == t_end) mbar_arrive(&kfull[ks]);   // pair without tile 1
+                } else if (KV8) {
+                    const uint32_t vs = it % NV;
+                    if (!mbar_wait_bounded(&vempty[vs], ((it / NV) & 1u) ^ 1u)) { alive = false; break; }
+                    if (m.nvalid > 0) {
+                        mbar_arrive_expect_tx(&v8full[vs], kTileBytes8);
+                        tma_load_3d(smem + L::kVOff + vs * kTileBytes + kHalfBytes, &vmap, &v8full[vs], 0, ty, tz, pol);
+                    } else {
+                        mbar_arrive(&v8full[vs]);
+                    }
                 } else {
                     const uint32_t vs = it % NV;
                     if (!mbar_wait_bounded(&vempty[vs], ((it / NV) & 1u) ^ 1u)) { alive = false; break; }
@@ -248,8 +329,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     } else if (warp == 1) {
         // =========================== S issuer (QK^T) =========================================
         if (lane == 0) {
-            constexpr uint32_t kIdescS64 = tc::idesc_bf16_f32(64, 64, false, false);
-            constexpr uint32_t kIdescS128 = tc::idesc_bf16_f32(64, 128, false, false);
+            constexpr uint32_t kIdescS64 = KV8 ? tc::idesc_f16_f32(64, 64, false, false)
+                                               : tc::idesc_bf16_f32(64, 64, false, false);
+            constexpr uint32_t kIdescS128 = KV8 ? tc::idesc_f16_f32(64, 128, false, false)
+                                                : tc::idesc_bf16_f32(64, 128, false, false);
+            uint64_t* q_ready = KV8 ? q_conv : q_full;   // fp8: Q widened to fp16 in place first
             // descriptors of the ring bases; a k-step or buffer offset is added as (bytes >> 4)
             const uint64_t dK = tc::smem_desc(smem_addr(smem + L::kKOff), 16, 1024);
             const uint64_t dQ = tc::smem_desc(smem_addr(smem + L::kQOff), 16, 1024);
@@ -265,7 +349,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 for (uint32_t sub = 0; sub < (has1 ? 2u : 1u); ++sub) {
                     mt[sub] = kmeta[2 * ks + sub];
                     if (mt[sub].flags & kFirst) {
-                        if (!mbar_wait_bounded(&q_full[uidx & 1u], (uidx >> 1) & 1u)) { ok = false; break; }
+                        if (!mbar_wait_bounded(&q_ready[uidx & 1u], (uidx >> 1) & 1u)) { ok = false; break; }
                         ++uidx;
                     }
                     qb[sub] = (uidx - 1u) & 1u;
@@ -312,15 +396,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     } else if (warp == 7) {
         // =========================== PV issuer ===============================================
         if (lane == 0) {
-            constexpr uint32_t kIdescO = tc::idesc_bf16_f32(64, 128, false, true);
+            constexpr uint32_t kIdescO = KV8 ? tc::idesc_f16_f32(64, 128, false, true)
+                                             : tc::idesc_bf16_f32(64, 128, false, true);
             const uint64_t dP = tc::smem_desc(smem_addr(smem + L::kPOff), 16, 1024);
             const uint64_t dV = tc::smem_desc(smem_addr(smem + L::kVOff), 8192, 1024);
             uint32_t o_init[2] = {0u, 0u};
             int o_unit[2] = {-1, -1};
             for (uint32_t t = 0; t < n; ++t) {
-                const uint32_t sb = t % kTcPBufs, vs = t % NV, g = t & 1u;
+                const uint32_t sb = t % kPB, vs = t % NV, g = t & 1u;
                 // the softmax group of tile t has written P(t) (and read its description) by now
-                if (!mbar_wait_bounded(&p_full[sb], (t / kTcPBufs) & 1u)) break;
+                if (!mbar_wait_bounded(&p_full[sb], (t / kPB) & 1u)) break;
                 const TileMeta m = pmeta[sb];
                 if (!mbar_wait_bounded(&vfull[vs], (t / NV) & 1u)) break;
                 tc::fence_after_sync();
@@ -339,6 +424,58 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             }
             tc::commit(&mma_done[1]);
             mbar_wait_bounded(&mma_done[1], 0);
+        }
+    } else if (KV8 && warp >= 12) {
+        // =========================== converters (fp8 KV) =====================================
+        // warps 12-13 widen each K tile in its pair slot (and each unit's Q rows to fp16 in
+        // place), warps 14-15 each V tile in its V slot; thread r owns key row r.  The MMAs read
+        // only fp16 operands.
+        const bool conv_k = warp < 14;
+        const int r = threadIdx.x - (conv_k ? 384 : 448);          // 0 .. 63
+        uint32_t uq = 0;
+        for (uint32_t t = 0; t < n; ++t) {
+            if (conv_k) {
+                const uint32_t pq = t >> 1, sub = t & 1u, ks = pq % NK;
+                if (!mbar_wait_bounded(&k8full[2 * ks + sub], (pq / NK) & 1u)) break;
+                const TileMeta m = kmeta[2 * ks + sub];
+                if (m.flags & kFirst) {
+                    const uint32_t qb = uq & 1u;
+                    if (!mbar_wait_bounded(&q_full[qb], (uq >> 1) & 1u)) break;
+                    const uint32_t qa = smem_addr(smem + L::kQOff + qb * L::kQBytes);
+                    for (int i = r; i < L::kQBytes / 16; i += 64) {
+                        uint32_t v0, v1, v2, v3;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3) : "r"(qa + 16u * i));
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(qa + 16u * i), "r"(bf16x2_to_f16x2(v0)), "r"(bf16x2_to_f16x2(v1)),
+                                        "r"(bf16x2_to_f16x2(v2)), "r"(bf16x2_to_f16x2(v3))
+                                     : "memory");
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&q_conv[qb]);
+                    ++uq;
+                }
+                if (m.nvalid > 0) {
+                    const uint32_t base = smem_addr(smem + L::kKOff + ks * L::kKSlotBytes + sub * kHalfBytes);
+                    widen_rows(base + kTileBytes, base, m.nvalid, r);
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&kfull[ks]);
+                    if (sub == 0u && t + 1 == n) mbar_arrive(&kfull[ks]);   // pair without tile 1
+                }
+            } else {
+                const uint32_t vs = t % NV;
+                if (!mbar_wait_bounded(&v8full[vs], (t / NV) & 1u)) break;
+                // rows past the valid keys come out as zeros (codes there may be anything)
+                const uint32_t base = smem_addr(smem + L::kVOff + vs * kTileBytes);
+                widen_rows(base + kHalfBytes, base, kTileKeys, r);
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vfull[vs]);
+            }
         }
     } else {
         // =========================== softmax warps (two groups) ==============================
@@ -362,7 +499,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         for (uint32_t it = grp; it < n && alive; it += 2) {
             const uint32_t sq = (it >> 1) % NSB;             // S pair buffer
             const uint32_t scol = sq * 128u + 64u * grp;     // this tile's 64 score columns
-            const uint32_t sb = it % kTcPBufs;               // P buffer
+            const uint32_t sb = it % kPB;                    // P buffer
             if (!mbar_wait_bounded(&s_full[sq], ((it >> 1) / NSB) & 1u)) { alive = false; break; }
             tc::fence_after_sync();
             const TileMeta m = smeta[2 * sq + grp];
@@ -438,12 +575,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             for (int j = 0; j < 16; ++j) {
                 const float p0 = fast_exp2(fmaf(x[2 * j], a.scale_log2, -m_sub));
                 const float p1 = fast_exp2(fmaf(x[2 * j + 1], a.scale_log2, -m_sub));
-                pk[j] = pack_bf16x2(p0, p1);
-                ls[j & 3] += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+                if (KV8) {
+                    // fp16 weights for the fp16 V; the row sum over the same rounded weights
+                    pk[j] = pack_f16x2(p0, p1);
+                    const float2 pr = __half22float2(*reinterpret_cast<const __half2*>(&pk[j]));
+                    ls[j & 3] += pr.x + pr.y;
+                } else {
+                    pk[j] = pack_bf16x2(p0, p1);
+                    ls[j & 3] += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+                }
             }
             l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             // ---- P to shared memory (its buffer is free once PV of tile it - NSB is done) -----
-            if (it >= (uint32_t)kTcPBufs && !mbar_wait_bounded(&p_free[sb], ((it / kTcPBufs) & 1u) ^ 1u)) {
+            if (it >= (uint32_t)kPB && !mbar_wait_bounded(&p_free[sb], ((it / kPB) & 1u) ^ 1u)) {
                 alive = false;
                 break;
             }
@@ -472,8 +616,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             //      previous PV, tile it - 2, is done) --------------------------------------------
             if (__any_sync(0xffffffffu, rescale)) {
                 if (it >= 2u) {
-                    const uint32_t pb = (it - 2u) % kTcPBufs;
-                    if (!mbar_wait_bounded(&p_free[pb], ((it - 2u) / kTcPBufs) & 1u)) { alive = false; break; }
+                    const uint32_t pb = (it - 2u) % kPB;
+                    if (!mbar_wait_bounded(&p_free[pb], ((it - 2u) / kPB) & 1u)) { alive = false; break; }
                 }
                 tc::fence_after_sync();
                 const float f = rescale ? alpha : 1.f;
@@ -505,15 +649,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             if (lane == 0) mbar_arrive(&p_full[sb]);
             // ---- unit end: combine both groups' (O, max, sum), write the rows ----------------
             if (m.flags & kLast) {
-                if (!mbar_wait_bounded(&p_free[sb], (it / kTcPBufs) & 1u)) { alive = false; break; }
+                if (!mbar_wait_bounded(&p_free[sb], (it / kPB) & 1u)) { alive = false; break; }
                 // the other group's last tile of this unit, if any, is tile it - 1: its P (and so
                 // its published state) is complete once its p_full phase has, and its PV before
                 // ours
                 bool other = false;
                 float m_o = -INFINITY, l_o = 0.f;
                 if (it >= 1u) {
-                    const uint32_t pb = (it - 1u) % kTcPBufs;
-                    if (!mbar_wait_bounded(&p_full[pb], ((it - 1u) / kTcPBufs) & 1u)) { alive = false; break; }
+                    const uint32_t pb = (it - 1u) % kPB;
+                    if (!mbar_wait_bounded(&p_full[pb], ((it - 1u) / kPB) & 1u)) { alive = false; break; }
                     if (pub_unit[grp ^ 1u] == m.unit) {
                         other = true;
                         m_o = pub_m_oth[row];
@@ -525,7 +669,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 const float w_own = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
                 const float w_oth = (!other || m_o == -INFINITY) ? 0.f : fast_exp2(m_o - M);
                 const float l_sum = l_row * w_own + l_o * w_oth;
-                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const float inv = l_sum > 0.f ? a.v_scale / l_sum : 0.f;
                 const float lse2 = l_sum > 0.f ? M + __log2f(l_sum) : -INFINITY;
                 const bool use_own = w_own > 0.f, use_oth = w_oth > 0.f;
                 const int R = m.rb * kRowsPerBlock + row;

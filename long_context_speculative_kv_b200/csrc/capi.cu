@@ -262,11 +262,11 @@ char tc_variant() {
 
 int tc_ctas_per_sm() { return 1; }
 
-template <int SRC, int NK, int NV, int NSB>
+template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
 int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
                      int sm_count, const Shape& s, cudaStream_t st) {
-    using Lay = TcLayout<NK, NV, NSB>;
-    auto kern = attn_tc_kernel<SRC, NK, NV, NSB>;
+    using Lay = TcLayout<NK, NV, NSB, KV8>;
+    auto kern = attn_tc_kernel<SRC, NK, NV, NSB, KV8>;
     static bool attr_set[kMaxDevices] = {};
     int dev;
     if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
@@ -279,7 +279,7 @@ int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q
     int rc = encode_q_map(&qm, q, s.B, s.n_q, s.Hq, s.Hkv);
     if (rc != WMTP_OK) return rc;
     const int grid = sm_count;
-    rc = launch(kern, dim3(grid), dim3(kTcThreads), Lay::kAlloc, st, km, vm, qm, a);
+    rc = launch(kern, dim3(grid), dim3(tc_threads<KV8>()), Lay::kAlloc, st, km, vm, qm, a);
     if (rc != WMTP_OK) return rc;
     return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
@@ -298,9 +298,31 @@ int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, 
 // throughout: widening the codes lengthens each warp's dependency chains, so the consumer warps
 // need the second CTA's warps to hide them (ncu on the one-CTA layout: 5 warps per SM, issue
 // slots 32 % busy, stalls mostly on fixed-latency dependencies).
+// fp8 units on the tcgen05 kernel (converter warps widen each tile once, in place, into fp16
+// operands): by default units of 33..64 rows, where the register-widening layouts redo the
+// work per m-tile warp (at 1M keys: 48 rows 441 vs 463 us, 64 rows 423 vs 566 us; 32 rows
+// 431 vs 345 us for the register path); WMTP_TC8=0 turns it off, WMTP_TC8=all uses it for every
+// unit of at most 64 rows.
+int tc8_mode() {
+    static int v = [] {
+        const char* e = std::getenv("WMTP_TC8");
+        if (e && e[0] == 'a') return 2;
+        if (e && e[0] == '0') return 0;
+        return 1;
+    }();
+    return v;
+}
+
+bool use_tc8(const Shape& s) {
+    if (s.rows_total > kRowsPerBlock) return false;
+    const int mode = tc8_mode();
+    return mode == 2 || (mode == 1 && s.rows_blk > 32);
+}
+
 template <int SRC>
 int launch_attn_kv8(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                     const Shape& s, cudaStream_t st) {
+    if (use_tc8(s)) return launch_attn_tc_t<SRC, 3, 3, 2, true>(km, vm, a.q, a, sm_count, s, st);
     switch ((s.rows_blk + 15) / 16) {
         case 1: return launch_attn_t<SRC, 1, 4, 4, 2, true>(km, vm, a, sm_count, s, st);
         case 2: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
@@ -345,7 +367,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
 
 // CTAs per SM of the variant a call with these rows will use.
 int ctas_per_sm_for(const Shape& s, bool kv8 = false) {
-    if (kv8) return 2;
+    if (kv8) return use_tc8(s) ? 1 : 2;
     if (use_tc(s)) return tc_ctas_per_sm();
     const int nmt = (s.rows_blk + 15) / 16;
     const char v = variant_for(nmt < 4 ? nmt : 4);
