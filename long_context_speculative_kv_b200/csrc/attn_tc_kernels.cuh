@@ -5,35 +5,42 @@
 // [128 x 64] contractions per key tile.
 //
 // Same work split, tile walk, masks, partial format and merge as attn_split_kernel; only the
-// math engine differs.  Roles (384 threads, one CTA per SM):
-//   warp 0        K producer: each tile's K (two 64x64 TMA boxes) into an NK-deep ring, and each
-//                 unit's Q rows (one box of n_q x G rows per 64-dim half) into a Q double buffer;
+// math engine differs.  Tiles go in pairs (CTA-local tiles 2q, 2q + 1).  Roles (384 threads, one
+// CTA per SM; 512 with fp8 KV):
+//   warp 0        K producer: each pair's K tiles into one pair slot of an NK-deep ring (laid
+//                 out so the 128 keys of a 64-dim half are consecutive rows), and each unit's Q
+//                 rows (one box of n_q x G rows per 64-dim half) into a Q double buffer;
 //   warp 6        V producer: each tile's V into an NV-deep ring.  K is released as soon as
-//                 QK^T has read it and V after PV, so K streams up to NK tiles ahead;
-//   warp 1        owns the tensor memory; lane 0 issues S[t % NSB] = Q K^T (tcgen05.mma,
-//                 M = 64 rows, N = 64 keys, K = 128, fp32 in TMEM) as soon as a K tile and an S
-//                 buffer are ready, and forwards each tile's description to the softmax warps
-//                 through the S barrier;
+//                 QK^T has read it and V after PV;
+//   warp 1        owns the tensor memory; lane 0 issues S = Q K^T for a pair into a 128-column
+//                 S buffer: one M = 64, N = 128, K = 16 MMA per k-step when both tiles belong to
+//                 the same unit, else two N = 64 sequences; fp32 in TMEM.  It forwards the tiles'
+//                 descriptions to the softmax warps through the S barrier;
 //   warp 7        lane 0 issues O += P V (M = 64, N = 128 dims, K = 64 keys; O stays in TMEM)
-//                 once the softmax warps have written P(t).  Two issuers keep the tensor core's
-//                 queue fed while the other waits;
+//                 into the tile's group's O once the softmax group has written P(t).  Two issuers
+//                 keep the tensor core's queue fed while the other waits;
 //   warps 2..5, 8..11   softmax, two groups of four warps taking alternate tiles (group g the
-//                 CTA's tiles it with it % 2 == g), each with its own running maxima and sums and
-//                 its own O accumulator in TMEM; one warp per sub-partition could not keep up
-//                 with the tile rate.  The M = 64 accumulator keeps row r in TMEM lane
-//                 32 (r / 16) + r % 16, so warp w sees rows 16 (w % 4) .. + 15; with the 16x32bx2
-//                 load both half-warps read those rows, lanes 0-15 keys 0-31 and lanes 16-31
-//                 keys 32-63 (and O dims 0-63 / 64-127).  Each thread masks, exponentiates against
-//                 the row's running maximum and writes its half of the P row (bf16, 128-byte
-//                 swizzled) for the PV MMA.  The maximum is only moved when a row's maximum grows
-//                 by more than 2^8 (log2 units), and only then is that O row rescaled in TMEM, so
-//                 the common tile touches no O at all.  After each tile a group publishes its
-//                 rows' maxima and sums; the group holding a unit's last tile combines both
-//                 groups' (O, max, sum) like two split-KV partials and writes the result, and a
-//                 group starts a new unit only after that combination (its O is then free).
-// Tensor memory: NSB S buffers of 64 columns, then O of group 0 and O of group 1 (128 columns
-// each).  Every wait is bounded; on a timeout all roles stop, each MMA issuer waits (bounded) for
-// its own MMAs, all meet at the final barrier and warp 1 frees the tensor memory.
+//                 CTA's tiles it with it % 2 == g, i.e. column half g of each S buffer), each with
+//                 its own running maxima and sums and its own O accumulator in TMEM; one warp per
+//                 sub-partition could not keep up with the tile rate.  The M = 64 accumulator
+//                 keeps row r in TMEM lane 32 (r / 16) + r % 16, so warp w sees rows
+//                 16 (w % 4) .. + 15; with the 16x32bx2 load both half-warps read those rows,
+//                 lanes 0-15 keys 0-31 and lanes 16-31 keys 32-63 (and O dims 0-63 / 64-127).
+//                 Each thread masks, exponentiates against the row's running maximum and writes
+//                 its half of the P row (128-byte swizzled) for the PV MMA.  The maximum is only
+//                 moved when a row's maximum grows by more than 2^8 (log2 units), and only then
+//                 is that O row rescaled in TMEM, so the common tile touches no O at all.  After
+//                 each tile a group publishes its rows' maxima and sums; the group holding a
+//                 unit's last tile combines both groups' (O, max, sum) like two split-KV partials
+//                 and writes the result, and a group starts a new unit only after that
+//                 combination (its O is then free);
+//   warps 12..15  (fp8 KV only) converters: each E4M3 tile lands in the upper half of its fp16
+//                 slot and is widened in place (two warps for K, two for V; eight warps measured
+//                 no faster); each unit's Q is widened bf16 -> fp16 in place.  The MMAs then
+//                 read fp16 operands only (P too).
+// Tensor memory: NSB S pair buffers of 128 columns, then O of group 0 and O of group 1 (128
+// columns each).  Every wait is bounded; on a timeout all roles stop, each MMA issuer waits
+// (bounded) for its own MMAs, all meet at the final barrier and warp 1 frees the tensor memory.
 #pragma once
 
 #include "attn_kernels.cuh"

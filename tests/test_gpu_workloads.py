@@ -5,7 +5,8 @@ Workloads: 128K context (GQA 16/2), 1M context (GQA 32/4), a ragged batch of 8 w
 rings and an 8-node draft tree, and 1M NoPE context (GQA 64/8) with 1% outlier rows across the
 window sweep 4 + {1020, 2044, 4092, 8188, 16380}.  The draft KV is appended to the rings by the
 library's own bulk append (only survivors are written) and paged into the pool for the full
-draft; the verify layer has its own paged KV holding the step's nodes.
+draft; the verify layer has its own paged KV holding the step's nodes.  The 1M workload also
+runs with every cache in fp8 (E4M3) codes.
 """
 import numpy as np
 import pytest
@@ -147,3 +148,90 @@ def test_batch8_ragged_tree():
 def test_nope1m_outliers_window_sweep():
     w = configs.NOPE1M
     _run_workload(w, 5, list(w.windows), _samples_factory([0, 7], w.G, n_rows=3))
+
+
+# ----------------------------------------------------------------------------- fp8 (E4M3) KV
+def _paginate8(tok, lens, table, num_pages, P):
+    """Token-major [B, Lmax, Hkv, D] codes -> pool [num_pages, Hkv, P, D]; rows past each
+    request's end hold the NaN code."""
+    B, Lmax, Hkv, D = tok.shape
+    pool = torch.full((num_pages, Hkv, P, D), 0x7F, dtype=torch.uint8, device=tok.device)
+    for b in range(B):
+        L = int(lens[b])
+        n_full = L // P
+        if n_full:
+            pages = torch.from_numpy(table[b, :n_full].astype(np.int64)).to(tok.device)
+            pool.index_copy_(0, pages, tok[b, :n_full * P].view(n_full, P, Hkv, D).permute(0, 2, 1, 3).contiguous())
+        r = L - n_full * P
+        if r:
+            pool[int(table[b, n_full]), :, :r] = tok[b, n_full * P:L].permute(1, 0, 2)
+    return pool
+
+
+def _sample_check8(out, lse, q_bits, k_tok, v_tok, L_tot, b, h, G, rows, mode, sm_scale, ks, vs, **kw):
+    kb = k_tok[b, :L_tot, h].contiguous().cpu().numpy().reshape(1, 1, L_tot, -1)
+    vb = v_tok[b, :L_tot, h].contiguous().cpu().numpy().reshape(1, 1, L_tot, -1)
+    qb = np.ascontiguousarray(q_bits[b:b + 1, :, h * G:(h + 1) * G])
+    ref, ref_lse = oracle.attention_kv8(qb, kb, vb, [L_tot], mode, sm_scale, ks, vs,
+                                        rows=[(0, i, g) for i, g in rows], **kw)
+    got = to_f64(out)
+    gl = lse.cpu().numpy()
+    a = np.stack([got[b, i, h * G + g] for i, g in rows])
+    r = np.stack([ref[0, i, g] for i, g in rows])
+    assert_attn_close(a, r, f"fp8 b{b} h{h}")
+    assert_lse_close(np.array([gl[b, i, h * G + g] for i, g in rows]),
+                     np.array([ref_lse[0, i, g] for i, g in rows]))
+
+
+def test_ctx1m_fp8_kv():
+    """The 1M workload with every cache in E4M3 codes: verify at 32 rows (register widening)
+    and 64 rows (tcgen05 with converter warps), the full draft, and the windowed draft over a
+    ring filled by the fp8 bulk append."""
+    w = configs.CTX1M
+    dev = "cuda"
+    KS, VS = 0.5, 0.5
+    L = w.L
+    G, P = w.G, w.page_size
+    g = tg.generator(w.seed + 77, dev)
+    samples = _samples_factory([0, 3], G, n_rows=3)
+    ws = api.alloc_workspace(1, 8, w.Hq, w.Hkv)
+    for gamma in (3, 7):
+        n_q = gamma + 1
+        Lv = L + n_q
+        k_t, v_t = tg.kv_rows_fp8((1, Lv, w.Hkv, w.D), g, dev)
+        table, npg = tg.page_table([Lv], P, w.seed + 1)
+        kp, vp = _paginate8(k_t, [Lv], table, npg, P), _paginate8(v_t, [Lv], table, npg, P)
+        q, q_bits = _q(g, 1, n_q, w.Hq, w.D)
+        out, lse = api.verify_attn_fp8(q, kp, vp, torch.from_numpy(table).cuda(),
+                                       torch.tensor([Lv], dtype=torch.int32, device=dev), w.sm_scale,
+                                       KS, VS, ws)
+        torch.cuda.synchronize()
+        assert api.device_status() == 0
+        for b, h, rows in samples(n_q):
+            _sample_check8(out, lse, q_bits, k_t, v_t, Lv, b, h, G, rows, oracle.MODE_CAUSAL, w.sm_scale, KS, VS)
+        del kp, vp
+    # draft: full over the paged cache, windowed over the ring (bulk fp8 append)
+    table, npg = tg.page_table([L], P, w.seed + 2)
+    kp, vp = _paginate8(k_t[:, :L], [L], table, npg, P), _paginate8(v_t[:, :L], [L], table, npg, P)
+    q, q_bits = _q(g, 1, 1, w.Hq, w.D)
+    out, lse = api.draft_attn_full_fp8(q, kp, vp, torch.from_numpy(table).cuda(),
+                                       torch.tensor([L], dtype=torch.int32, device=dev), w.sm_scale, KS, VS, ws)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    for b, h, rows in samples(1):
+        _sample_check8(out, lse, q_bits, k_t, v_t, L, b, h, G, rows, oracle.MODE_CAUSAL, w.sm_scale, KS, VS)
+    del kp, vp
+    W = w.windows[0]
+    C = w.n_sink + W
+    ring_k = torch.full((1, w.Hkv, C, w.D), 0x7F, dtype=torch.uint8, device=dev)
+    ring_v = ring_k.clone()
+    rlen = torch.zeros(1, dtype=torch.int64, device=dev)
+    api.ring_kv_append_fp8(ring_k, ring_v, rlen, k_t[:, :L].contiguous(), v_t[:, :L].contiguous(), w.n_sink)
+    for nq in (1, 4):
+        q, q_bits = _q(g, 1, nq, w.Hq, w.D)
+        out, lse = api.draft_attn_window_fp8(q, ring_k, ring_v, rlen, w.n_sink, W, w.sm_scale, KS, VS, ws)
+        torch.cuda.synchronize()
+        assert api.device_status() == 0
+        for b, h, rows in samples(nq):
+            _sample_check8(out, lse, q_bits, k_t, v_t, L, b, h, G, rows, oracle.MODE_WINDOW, w.sm_scale,
+                           KS, VS, n_sink=w.n_sink, window=W)
