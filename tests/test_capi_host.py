@@ -17,7 +17,11 @@ def lib():
 
 
 def _headers_src():
-    return "\n".join(open(h).read() for h in _lib.HEADERS)
+    parts = []
+    for h in _lib.HEADERS:
+        with open(h) as f:
+            parts.append(f.read())
+    return "\n".join(parts)
 
 
 def _declared():

@@ -81,7 +81,8 @@ PINS = [
 
 @pytest.mark.parametrize("name,orig,mut", MUTATIONS, ids=[m[0] for m in MUTATIONS])
 def test_pins_catch_planted_mistake(name, orig, mut):
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(orig) == 1, f"mutation anchor not unique: {orig!r}"
     with tempfile.TemporaryDirectory() as d:
         c = os.path.join(d, "mut.c")

@@ -32,7 +32,7 @@ def _worker(rank: int, world: int, port: int, out):
 def test_max_over_ranks_and_aggregate_with_two_gloo_ranks():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
