@@ -3,7 +3,8 @@
 Source: Pith verdict on arXiv 2607.21535, pith_extraction.forward_implications[4] (windowing
 composes with fp8 KV quantisation).  Codes come from N(0, 2^2) values rounded to E4M3; key and
 value scales are not powers of two; page tails hold NaN codes and unwritten ring slots hold
-garbage, so a stray read shows.  Row counts 8, 32, 48 and 64 per unit exercise every fp8 layout.
+garbage, so a stray read shows.  Row counts 8, 24, 25, 32, 48 and 64 per unit exercise every
+fp8 layout.
 """
 import numpy as np
 import pytest
@@ -79,6 +80,8 @@ def test_draft_full_fp8_matches_oracle(lens, Hq, Hkv, n_q):
 
 @pytest.mark.parametrize("lens,Hq,Hkv,n_q", [
     ([5000], 32, 4, 4),                      # gamma 3: 32 rows
+    ([64, 2047, 9000], 16, 2, 3),            # 24 rows: a ragged second m-tile
+    ([5, 300], 20, 4, 5),                    # 25 rows; the first request holds only the step
     ([777, 2500], 16, 2, 6),                 # 48 rows
     ([4100], 16, 2, 8),                      # 64 rows
 ])
@@ -91,12 +94,16 @@ def test_verify_chain_fp8_matches_oracle(lens, Hq, Hkv, n_q):
     assert_lse_close(lse, ref_lse, "verify_attn_fp8 chain lse")
 
 
-def test_verify_tree_fp8_matches_oracle():
+@pytest.mark.parametrize("Hq,Hkv,n_q", [
+    (32, 4, 8),                              # 64 rows
+    (32, 4, 4),                              # 32 rows
+])
+def test_verify_tree_fp8_matches_oracle(Hq, Hkv, n_q):
     sc = 128 ** -0.5
     lens = [900, 3000, 70]
-    c = paged8_case(13, lens, 32, 4, 8)
+    c = paged8_case(13, lens, Hq, Hkv, n_q)
     rng = np.random.default_rng(13)
-    tree = np.stack([gen.draft_tree(rng, 8) for _ in lens])
+    tree = np.stack([gen.draft_tree(rng, n_q) for _ in lens])
     out, lse = run_paged8(c, "verify", sc, tree=tree)
     ref, ref_lse = oracle.attention_kv8(c["q"], c["k8"], c["v8"], c["lens"], oracle.MODE_TREE, sc, KS, VS,
                                         tree_parent=tree)
