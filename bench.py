@@ -357,6 +357,50 @@ def run_gpu(args):
         assert api.device_status() == 0
         kernels["accept_stochastic"] = kstat([a.elapsed_time(c) for a, c in ev[5:]], 2 * w.B * w.vocab * 4)
 
+    # ---- device-side phase and small-call times: calls captured back to back in one CUDA graph
+    #      and replayed (as the step runs), so the host's issue time between eager calls, which
+    #      exceeds the device time of the small calls, is not counted ---------------------------
+    def graph_call_us(calls, replays):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for c in calls:
+                c()
+        torch.cuda.current_stream().wait_stream(side)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for c in calls:
+                c()
+        gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(replays):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del gr
+        return e0.elapsed_time(e1) * 1e3 / (replays * len(calls))
+
+    phases_graph, kernels_graph = None, {}
+    if use_graph:
+        Kp = max(5, args.steps // 10)
+        b_ = step.b
+        phases_graph = {
+            "windowed_t_draft_us": round(graph_call_us([step.draft_windowed], Kp), 2),
+            "native_t_draft_us": round(graph_call_us([step.draft_native], Kp), 2),
+            "t_verify_us": round(graph_call_us([step.verify], Kp), 2),
+            "t_accept_us": round(graph_call_us([step.accept] * 10, Kp), 2),
+        }
+        win_us = graph_call_us([lambda: step._window(b_.q_fwd[0], b_.out["fwd"], b_.out["fwd_lse"])] * 20, Kp)
+        app_us = graph_call_us([lambda: step._append(b_.k_fwd[0], b_.v_fwd[0])] * 20, Kp)
+        kernels_graph = {
+            "draft_attn_window_fwd": kstat([win_us / 1e3], bytes_window),
+            "ring_kv_append_1": kstat([app_us / 1e3], acc.append_bytes(1, w.Hkv, w.D) * w.B),
+            "accept_greedy": kstat([phases_graph["t_accept_us"] / 1e3], w.B * n_q_v * w.vocab * 4),
+        }
+        assert api.device_status() == 0
+
     # ---- windowed draft with a cold L2: rotate over ring copies larger than 2x L2 ----------
     cold = None
     if "ring_k" in shared:
@@ -380,6 +424,13 @@ def run_gpu(args):
         t = [a.elapsed_time(c) for a, c in times[R:]]
         cold = kstat(t, bytes_window)
         cold["rotating_copies"] = R
+        if use_graph:
+            def win_call(rk, rv):
+                return lambda: api.draft_attn_window(b.q_fwd[0], rk, rv, rl, w.n_sink, window, w.sm_scale,
+                                                     b.ws, out=b.out["fwd"], lse=b.out["fwd_lse"])
+            cold_us = graph_call_us([win_call(rk, rv) for rk, rv in rings], 3)
+            kernels_graph["draft_attn_window_fwd_cold"] = dict(kstat([cold_us / 1e3], bytes_window),
+                                                               rotating_copies=R)
         del rings
         torch.cuda.empty_cache()
 
@@ -604,9 +655,16 @@ def run_gpu(args):
 
     traffic = committed_traffic("verify_attn", w.name)
     v = kernels["verify_attn"]
+    v_src = "eager verify calls with CUDA events between calls"
+    if phases_graph:
+        # the step's verify layers as they run in the step's graph: back to back, each the
+        # attention kernel plus its LSE merge; per-layer mean of the replayed graph
+        v = kstat([phases_graph["t_verify_us"] / n_layers / 1e3], bytes_verify)
+        kernels_graph["verify_attn"] = v
+        v_src = "CUDA events around a graph of the step's verify layers, replayed; mean per layer"
     roofline = {"kernel": "verify_attn (split attention + LSE merge, one target layer)",
                 "bound": "hbm", "achieved": v["GBps"], "peak": hbm, "unit": "GB/s",
-                "frac": v["frac_of_hbm_peak"],
+                "frac": v["frac_of_hbm_peak"], "us_per_launch": v["us"], "duration_source": v_src,
                 "traffic": traffic, "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
 
@@ -630,6 +688,10 @@ def run_gpu(args):
         "native": {"us_per_step": round(us_n_local, 2), "us_per_step_eager": round(ms_n_eager * 1e3 / args.steps, 2),
                    "t_draft_us": round(tdn, 2), "t_verify_us": round(tvn, 2), "t_accept_us": round(tan, 2)},
         "phase_times_from": "eager launches with CUDA events between calls",
+        "phases_graph": phases_graph,
+        "kernels_graph": kernels_graph or None,
+        "kernels_graph_note": "each phase or call captured back to back in a CUDA graph and replayed; "
+                              "device time without the host issue gaps of eager calls",
         "step_cost_ratio_native_over_windowed": round(ms_n_max / ms_w_max, 4),
         "step_cost_reduction_pct": round(100 * (ms_n_max / ms_w_max - 1), 2),
         "kernels": dict(kernels, draft_attn_window_fwd_cold=cold),
