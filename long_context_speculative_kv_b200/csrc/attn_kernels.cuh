@@ -250,14 +250,23 @@ __device__ __forceinline__ unsigned long long step_visibility(const AttnArgs& a,
 
 // ---------------------------------------------------------------------------------------------
 // Shared-memory layout (dynamic; stage buffers 1024-byte aligned for the 128-byte swizzle).
-template <int NMT, int NKG, int NSTAGE, bool KV8 = false>
+// QS (fp8 KV only): the unit's Q rows are kept in shared memory as fp16, in a space the unit-end
+// key-group merge reuses one m-tile at a time.
+template <int NMT, int NKG, int NSTAGE, bool KV8 = false, bool QS = false>
 struct SmemLayout {
     static constexpr int kStagesBytes = NSTAGE * (KV8 ? kStageBytes8 : kStageBytes);
     static constexpr int kMergeStride = kD + 4;                      // floats per merge row
-    static constexpr int kMergeFloats = (NKG - 1) * NMT * 16 * kMergeStride;
-    static constexpr int kMergeMLFloats = (NKG - 1) * NMT * 16 * 2;
+    static constexpr int kMergeMT = QS ? 1 : NMT;                    // m-tiles merged at once
+    static constexpr int kMergeFloats = (NKG - 1) * kMergeMT * 16 * kMergeStride;
+    static constexpr int kMergeMLFloats = (NKG - 1) * kMergeMT * 16 * 2;
+    // fp16 Q row: 128 dims + 32 bytes of padding, so the 8-byte fragment reads of four rows in a
+    // half-warp start 8 banks apart
+    static constexpr int kQStride = 2 * kD + 32;
+    static constexpr int kQBytes = QS ? NMT * 16 * kQStride : 0;
     static constexpr int kMergeOff = kStagesBytes;
-    static constexpr int kMergeMLOff = kMergeOff + kMergeFloats * 4;
+    static constexpr int kQOff = kMergeOff;                          // QS: aliases the merge rows
+    static constexpr int kMergeBytes = (kQBytes > kMergeFloats * 4) ? kQBytes : kMergeFloats * 4;
+    static constexpr int kMergeMLOff = kMergeOff + kMergeBytes;
     static constexpr int kBarOff = kMergeMLOff + kMergeMLFloats * 4;
     static constexpr int kMetaOff = kBarOff + (2 * NSTAGE + 1) * 8;
     static constexpr int kPlanOff = kMetaOff + NSTAGE * (int)sizeof(TileMeta);
@@ -285,11 +294,16 @@ __device__ __forceinline__ uint32_t tile8_chunk_addr(uint32_t base, int row, int
 // key, so the MMA's k index is permuted consistently in Q (loaded in the same order) and K.
 // PV: the widened V fragments are transposed in registers (movmatrix), which permutes the
 // output's head dims in a fixed way that the final store undoes.
-template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false>
+//
+// QS = true (fp8 only) keeps the unit's Q in shared memory as fp16 instead of in registers: each
+// A fragment is read per k-step, the kernel fits in 128 registers, and three CTAs share an SM
+// (the fp8 kernel is bound by per-warp dependency chains, so more warps per SM is what helps).
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
 __global__ void __launch_bounds__((NMT * NKG + 1) * 32, MINB)
 attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const AttnArgs a) {
-    using L = SmemLayout<NMT, NKG, NSTAGE, KV8>;
+    using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
+    static_assert(!QS || KV8, "shared-memory Q is an fp8-KV layout");
     constexpr int kStage = KV8 ? kStageBytes8 : kStageBytes;
     constexpr int NWC = NMT * NKG;            // consumer warps
     constexpr int KPW = kTileKeys / NKG;      // keys per consumer warp per tile
@@ -445,6 +459,39 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             }
 #pragma unroll
             for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            if constexpr (QS) {
+                // every warp is past the previous unit's reads of these rows; each consumer thread
+                // widens quarter rows (32 dims) of the unit's Q into shared memory
+                if (!consumers_sync()) { alive = false; break; }
+                for (int w = threadIdx.x; w < NMT * 16 * 4; w += NWC * 32) {
+                    const int row = w >> 2, part = w & 3;
+                    const int R = m.rb * kRowsPerBlock + row;
+                    uint32_t h[16];
+                    if (R < a.rows_total) {
+                        const int i = R / a.G, g = R - (R / a.G) * a.G;
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD + 32 * part);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint4 v = __ldg(src + k);
+                            h[4 * k] = bf16x2_to_f16x2(v.x);
+                            h[4 * k + 1] = bf16x2_to_f16x2(v.y);
+                            h[4 * k + 2] = bf16x2_to_f16x2(v.z);
+                            h[4 * k + 3] = bf16x2_to_f16x2(v.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) h[k] = 0u;
+                    }
+                    const uint32_t dst = smem_addr(smem + L::kQOff) + (uint32_t)(row * L::kQStride + 64 * part);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(dst + 16u * k), "r"(h[4 * k]), "r"(h[4 * k + 1]),
+                                        "r"(h[4 * k + 2]), "r"(h[4 * k + 3]) : "memory");
+                }
+                if (!consumers_sync()) { alive = false; break; }
+            } else {
             const uint32_t* q32[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
@@ -474,6 +521,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     qa[ks][3] = row_ok[1] ? __ldg(q32[1] + c + 4) : 0u;
                 }
             }
+            }
         }
 
         if (m.nvalid > 0) {
@@ -489,6 +537,23 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 const int c8 = lane >> 4;
 #pragma unroll
                 for (int kp = 0; kp < 4; ++kp) {
+                    // A fragments of k-steps 2 kp, 2 kp + 1 (QS: from the shared fp16 rows, dims
+                    // 16 ks + 4 tig .. + 3 of rows gid and gid + 8)
+                    uint32_t qs[2][4];
+                    if constexpr (QS) {
+#pragma unroll
+                        for (int kss = 0; kss < 2; ++kss) {
+                            const uint32_t q0 = smem_addr(smem + L::kQOff) +
+                                                (uint32_t)((mt * 16 + gid) * L::kQStride + 32 * (2 * kp + kss) + 8 * tig);
+                            const uint32_t q1 = q0 + 8u * L::kQStride;
+                            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                         : "=r"(qs[kss][0]), "=r"(qs[kss][2]) : "r"(q0));
+                            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                         : "=r"(qs[kss][1]), "=r"(qs[kss][3]) : "r"(q1));
+                        }
+                    }
+                    const uint32_t* A0 = QS ? qs[0] : qa[2 * kp];
+                    const uint32_t* A1 = QS ? qs[1] : qa[2 * kp + 1];
 #pragma unroll
                     for (int np = 0; np < NT / 2; ++np) {
                         uint32_t r0, r1, r2, r3;
@@ -498,10 +563,10 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         e4m3x4_to_f16x2x2(r1, b[2], b[3]);
                         e4m3x4_to_f16x2x2(r2, b[4], b[5]);
                         e4m3x4_to_f16x2x2(r3, b[6], b[7]);
-                        mma_f16_16816(s[2 * np], qa[2 * kp], b[0], b[1]);
-                        mma_f16_16816(s[2 * np + 1], qa[2 * kp], b[2], b[3]);
-                        mma_f16_16816(s[2 * np], qa[2 * kp + 1], b[4], b[5]);
-                        mma_f16_16816(s[2 * np + 1], qa[2 * kp + 1], b[6], b[7]);
+                        mma_f16_16816(s[2 * np], A0, b[0], b[1]);
+                        mma_f16_16816(s[2 * np + 1], A0, b[2], b[3]);
+                        mma_f16_16816(s[2 * np], A1, b[4], b[5]);
+                        mma_f16_16816(s[2 * np + 1], A1, b[6], b[7]);
                     }
                 }
             } else {
@@ -644,7 +709,54 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 1);
                 l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 2);
             }
-            if (NKG > 1) {
+            if (QS && NKG > 1) {
+                // one m-tile at a time through the shared Q rows' space, once every warp is past
+                // its last reads of them
+                if (!consumers_sync()) { alive = false; break; }
+#pragma unroll 1
+                for (int mt2 = 0; mt2 < NMT; ++mt2) {
+                    if (mt == mt2 && kg > 0) {
+                        float* mo = merge_o + ((size_t)(kg - 1) * 16) * L::kMergeStride;
+                        float* ml = merge_ml + ((size_t)(kg - 1) * 16) * 2;
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int row = gid + 8 * r;
+#pragma unroll
+                            for (int n = 0; n < 16; ++n)
+                                *reinterpret_cast<float2*>(mo + row * L::kMergeStride + n * 8 + 2 * tig) =
+                                    make_float2(o[n][2 * r], o[n][2 * r + 1]);
+                            if (tig == 0) { ml[row * 2] = m_r[r]; ml[row * 2 + 1] = l_r[r]; }
+                        }
+                    }
+                    if (!consumers_sync()) { alive = false; break; }
+                    if (mt == mt2 && kg == 0) {
+#pragma unroll 1
+                        for (int g2 = 1; g2 < NKG; ++g2) {
+                            const float* mo = merge_o + ((size_t)(g2 - 1) * 16) * L::kMergeStride;
+                            const float* ml = merge_ml + ((size_t)(g2 - 1) * 16) * 2;
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                const int row = gid + 8 * r;
+                                const float m2 = ml[row * 2], l2 = ml[row * 2 + 1];
+                                const float mn = fmaxf(m_r[r], m2);
+                                const float mu = (mn == -INFINITY) ? 0.f : mn;
+                                const float w1 = fast_exp2(m_r[r] - mu), w2 = fast_exp2(m2 - mu);
+                                l_r[r] = l_r[r] * w1 + l2 * w2;
+                                m_r[r] = mn;
+#pragma unroll
+                                for (int n = 0; n < 16; ++n) {
+                                    const float2 v2 = *reinterpret_cast<const float2*>(
+                                        mo + row * L::kMergeStride + n * 8 + 2 * tig);
+                                    o[n][2 * r] = o[n][2 * r] * w1 + v2.x * w2;
+                                    o[n][2 * r + 1] = o[n][2 * r + 1] * w1 + v2.y * w2;
+                                }
+                            }
+                        }
+                    }
+                    if (!consumers_sync()) { alive = false; break; }
+                }
+                if (!alive) break;
+            } else if (NKG > 1) {
                 if (kg > 0) {
                     float* mo = merge_o + ((size_t)((kg - 1) * NMT + mt) * 16) * L::kMergeStride;
                     float* ml = merge_ml + ((size_t)((kg - 1) * NMT + mt) * 16) * 2;

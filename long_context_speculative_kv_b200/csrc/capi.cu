@@ -198,7 +198,7 @@ int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStrea
 //   rows 32: A (2, 2, 2 CTAs) 0.97 | (2, 4, 1) 0.81 | (1, 3, 2) 0.82
 //   rows 48: A (1, 2, 2) 0.81 | (1, 3, 2) 0.81 | (2, 4, 1) 0.70
 //   rows 64: A (1, 2, 2) 0.66 | (1, 3, 2) 0.65 | (2, 4, 1) 0.52
-constexpr int kMaxCtasPerSm = 2;
+constexpr int kMaxCtasPerSm = 3;
 
 char variant_for(int nmt) {
     static char v[5] = {0, 0, 0, 0, 0};
@@ -211,11 +211,11 @@ char variant_for(int nmt) {
     return v[nmt];
 }
 
-template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false>
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
 int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                   const Shape& s, cudaStream_t st) {
-    using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8>;
-    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB, KV8>;
+    using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
+    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB, KV8, QS>;
     static bool attr_set[kMaxDevices] = {};
     int dev;
     if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
@@ -319,10 +319,29 @@ bool use_tc8(const Shape& s) {
     return mode == 2 || (mode == 1 && s.rows_blk > 32);
 }
 
+// fp8 units with Q in shared memory and three CTAs per SM: by default units of at most 16
+// rows (the one-query draft at 1M keys: 199 vs 216 us); at 17..32 rows it measured no faster
+// (347 vs 344 us) and the two-CTA register layout stays.  WMTP_FP8QS=0 turns it off,
+// WMTP_FP8QS=all uses it up to 32 rows (sweeps).
+bool use_fp8qs(const Shape& s) {
+    static int v = [] {
+        const char* e = std::getenv("WMTP_FP8QS");
+        if (e && e[0] == 'a') return 2;
+        if (e && e[0] == '0') return 0;
+        return 1;
+    }();
+    if (use_tc8(s)) return false;
+    return (v == 1 && s.rows_blk <= 16) || (v == 2 && s.rows_blk <= 32);
+}
+
 template <int SRC>
 int launch_attn_kv8(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                     const Shape& s, cudaStream_t st) {
     if (use_tc8(s)) return launch_attn_tc_t<SRC, 3, 3, 2, true>(km, vm, a.q, a, sm_count, s, st);
+    if (use_fp8qs(s)) {
+        if (s.rows_blk <= 16) return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);
+        return launch_attn_t<SRC, 2, 2, 3, 3, true, true>(km, vm, a, sm_count, s, st);
+    }
     switch ((s.rows_blk + 15) / 16) {
         case 1: return launch_attn_t<SRC, 1, 4, 4, 2, true>(km, vm, a, sm_count, s, st);
         case 2: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
@@ -367,7 +386,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
 
 // CTAs per SM of the variant a call with these rows will use.
 int ctas_per_sm_for(const Shape& s, bool kv8 = false) {
-    if (kv8) return use_tc8(s) ? 1 : 2;
+    if (kv8) return use_tc8(s) ? 1 : (use_fp8qs(s) ? 3 : 2);
     if (use_tc(s)) return tc_ctas_per_sm();
     const int nmt = (s.rows_blk + 15) / 16;
     const char v = variant_for(nmt < 4 ? nmt : 4);
