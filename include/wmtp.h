@@ -271,8 +271,18 @@ WMTP_API int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring
 WMTP_API uint64_t wmtp_launch_count(void);
 
 /* Reads and clears the device status word on the current device (synchronizes `stream`).
- * Returns WMTP_OK, WMTP_ERR_DEVICE_INDEX, or WMTP_ERR_CUDA if the read itself failed. */
+ * Returns WMTP_OK, WMTP_ERR_DEVICE_INDEX, WMTP_ERR_TIMEOUT, or WMTP_ERR_CUDA if the read itself
+ * failed. */
 WMTP_API int wmtp_device_status(wmtp_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * wmtp_selftest_wait_timeout -- exercises the library's failure path without a fault (not part
+ * of the method).  Launches one CTA whose thread waits on a shared-memory mbarrier that nothing
+ * arrives on, with the same bounded spin the kernels use but a limit of `limit_ns` nanoseconds
+ * (1 ms .. 2 s); it then sets the timeout bit of the device status word and returns, so the next
+ * wmtp_device_status reports WMTP_ERR_TIMEOUT and the context stays usable.
+ *   Errors: WMTP_ERR_ARG for a limit outside [1e6, 2e9] ns; WMTP_ERR_CUDA for a launch failure. */
+WMTP_API int wmtp_selftest_wait_timeout(uint64_t limit_ns, wmtp_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -161,6 +161,12 @@ def device_status(stream=None) -> int:
     return int(lib().wmtp_device_status(_stream(stream)))
 
 
+def selftest_wait_timeout(limit_ns: int = 50_000_000, stream=None) -> None:
+    """Runs the library's bounded-wait failure path on purpose (a wait nothing satisfies); the
+    next device_status() returns WMTP_ERR_TIMEOUT."""
+    check("wmtp_selftest_wait_timeout", lib().wmtp_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
 def launch_count() -> int:
     """Kernels the library has launched in this process so far."""
     return int(lib().wmtp_launch_count())

@@ -491,6 +491,25 @@ int noalloc_scratch(void** out) {
 
 using namespace wmtp;
 
+// The failure path of every bounded wait, on purpose: lane 0 waits on an mbarrier that nothing
+// arrives on, gives up after limit_ns, flags the timeout status and returns (no trap, no fault).
+__global__ void selftest_wait_timeout_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        const uint64_t t0 = global_ns();
+        uint32_t spins = 0;
+        while (!mbar_try_wait(&bar, 0u)) {
+            if ((++spins & 255u) == 0u && global_ns() - t0 > limit_ns) {
+                flag_status(kStatusTimeout);
+                break;
+            }
+        }
+    }
+    __syncwarp();
+}
+
 extern "C" {
 
 const char* wmtp_status_string(int status) {
@@ -795,6 +814,12 @@ int wmtp_synth_target_logits(const int32_t* history, const int64_t* n_tokens, in
 }
 
 uint64_t wmtp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int wmtp_selftest_wait_timeout(uint64_t limit_ns, wmtp_stream_t stream) {
+    if (limit_ns < 1000000ull || limit_ns > kWaitLimitNs) return WMTP_ERR_ARG;
+    return launch(selftest_wait_timeout_kernel, dim3(1), dim3(32), 0,
+                  reinterpret_cast<cudaStream_t>(stream), limit_ns);
+}
 
 int wmtp_device_status(wmtp_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return WMTP_ERR_CUDA;

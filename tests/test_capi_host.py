@@ -35,7 +35,7 @@ def test_header_declares_the_five_calls_and_helpers():
             "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc",
             "accept_stochastic", "ring_kv_append_at", "spec_commit", "ring_kv_append_fp8",
             "draft_attn_window_fp8", "draft_attn_full_fp8", "verify_attn_fp8", "wmtp_synth_draft_tokens",
-            "wmtp_synth_target_logits"} == names
+            "wmtp_synth_target_logits", "wmtp_selftest_wait_timeout"} == names
     assert set(_lib._SIGNATURES) == names
 
 
@@ -96,6 +96,13 @@ def test_attention_host_checks(lib):
     v = lib.verify_attn
     assert v(GOOD, GOOD, GOOD, GOOD, GOOD, BAD, 1, 4, 8, 2, 128, 64, 4, 4, 1.0, GOOD, None, GOOD, 1 << 30, None) == -3
     assert v(GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, 4, 8, 2, 128, 64, 4, 4, 1.0, GOOD, None, GOOD, 1 << 30, None) == -1
+
+
+def test_selftest_wait_limit_checked_on_host(lib):
+    f = lib.wmtp_selftest_wait_timeout
+    assert f(999_999, None) == -1                 # below 1 ms
+    assert f(2_000_000_001, None) == -1           # above the kernels' own 2 s limit
+    assert f(0, None) == -1
 
 
 def test_accept_host_checks(lib):

@@ -286,3 +286,19 @@ def test_rising_scores_move_the_running_maximum(n_q, Hq, Hkv, tree):
     ref, ref_lse = oracle.attention(q, k, v, c["lens"], mode, sc, tree_parent=parent)
     assert_attn_close(out, ref, "rising scores")
     assert_lse_close(lse, ref_lse)
+
+
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """The failure path every kernel wait shares, on purpose: a wait that nothing satisfies gives
+    up after its limit, the status word reports WMTP_ERR_TIMEOUT (read and cleared), and the next
+    call on the same context still matches the oracle."""
+    assert api.device_status() == 0
+    api.selftest_wait_timeout(20_000_000)                # 20 ms
+    assert api.device_status() == -8                     # WMTP_ERR_TIMEOUT
+    assert api.device_status() == 0
+    sc = 128 ** -0.5
+    c = paged_case(7, [300, 1000], 8, 2, 1)
+    out, lse = run_paged(c, "full", sc)
+    ref, ref_lse = oracle.attention(c["q"], c["k"], c["v"], c["lens"], oracle.MODE_CAUSAL, sc)
+    assert_attn_close(out, ref)
+    assert_lse_close(lse, ref_lse)

@@ -166,3 +166,36 @@ def test_fp8_equals_bf16_path_on_identical_values():
     ref, _ = oracle.attention_kv8(c["q"], c["k8"], c["v8"], c["lens"], oracle.MODE_CAUSAL, sc, 1.0, 1.0)
     assert_attn_close(to_f64(o8), ref, "fp8 path")
     assert_attn_close(to_f64(o16), ref, "bf16 path")
+
+
+@pytest.mark.parametrize("Hq,Hkv,n_q", [
+    (8, 2, 1),                               # 4 rows: shared-memory Q layout
+    (8, 2, 4),                               # 16 rows: shared-memory Q layout, 4 queries
+    (32, 4, 4),                              # 32 rows: register layout
+])
+def test_fp8_empty_and_short_sequences(Hq, Hkv, n_q):
+    """kv_len 0 gives out 0 / lse -inf; kv_len < n_q leaves the early queries with no keys."""
+    sc = 0.1
+    c = paged8_case(15, [0, 2, 70], Hq, Hkv, n_q)
+    out, lse = run_paged8(c, "full", sc)
+    ref, ref_lse = oracle.attention_kv8(c["q"], c["k8"], c["v8"], c["lens"], oracle.MODE_CAUSAL, sc, KS, VS)
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert_attn_close(out, ref, "draft_attn_full_fp8 short")
+    assert_lse_close(lse, ref_lse, "draft_attn_full_fp8 short lse")
+
+
+def test_fp8_bad_page_id_sets_status_and_skips_tile():
+    sc = 128 ** -0.5
+    c = paged8_case(16, [640, 640], 8, 2, 1)
+    bad = c["table"].copy()
+    bad[1, 3] = 10 ** 6                                  # out of range for request 1 only
+    B, n_q, Hq, _ = c["q"].shape
+    ws = api.alloc_workspace(B, n_q, Hq, 2)
+    out, _ = api.draft_attn_full_fp8(to_dev_bf16(c["q"]), dev8(c["kp"]), dev8(c["vp"]),
+                                     torch.from_numpy(bad).cuda(),
+                                     torch.from_numpy(c["lens"].astype(np.int32)).cuda(), sc, KS, VS, ws)
+    assert api.device_status() == -6
+    assert api.device_status() == 0                      # read-and-clear
+    ref, _ = oracle.attention_kv8(c["q"], c["k8"], c["v8"], c["lens"], oracle.MODE_CAUSAL, sc, KS, VS)
+    assert_attn_close(to_f64(out)[:1], ref[:1], "request 0 unaffected")
+    assert not np.isnan(to_f64(out)).any()
