@@ -15,6 +15,7 @@
 #include "wmtp_loop.h"
 #include "attn_kernels.cuh"
 #include "attn_tc_kernels.cuh"
+#include "attn_tct_kernels.cuh"
 #include "ring_accept_kernels.cuh"
 #include "loop_kernels.cuh"
 #include "synth_kernels.cuh"
@@ -284,6 +285,46 @@ int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q
     return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
 
+// Units of at most 32 rows on the transposed tcgen05 kernel: WMTP_TCT=1 for 17..32 rows,
+// WMTP_TCT=all for every unit of at most 32 rows (bf16 and fp8 KV).
+int tct_mode() {
+    static int v = [] {
+        const char* e = std::getenv("WMTP_TCT");
+        if (e && e[0] == 'a') return 2;
+        if (e && e[0] == '1') return 1;
+        return 0;
+    }();
+    return v;
+}
+
+bool use_tct(const Shape& s) {
+    if (s.rows_total > kTctRows) return false;
+    const int mode = tct_mode();
+    return mode == 2 || (mode == 1 && s.rows_blk > 16);
+}
+
+template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
+int launch_attn_tct_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
+                      int sm_count, const Shape& s, cudaStream_t st) {
+    using Lay = TctLayout<NK, NV, NSB, KV8>;
+    auto kern = attn_tct_kernel<SRC, NK, NV, NSB, KV8>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev;
+    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess)
+            return WMTP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    CUtensorMap qm;
+    int rc = encode_q_map(&qm, q, s.B, s.n_q, s.Hq, s.Hkv);
+    if (rc != WMTP_OK) return rc;
+    const int grid = sm_count;
+    rc = launch(kern, dim3(grid), dim3(tct_threads<KV8>()), Lay::kAlloc, st, km, vm, qm, a);
+    if (rc != WMTP_OK) return rc;
+    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
+}
+
 template <int SRC>
 int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
                    int sm_count, const Shape& s, cudaStream_t st) {
@@ -338,6 +379,7 @@ template <int SRC>
 int launch_attn_kv8(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                     const Shape& s, cudaStream_t st) {
     if (use_tc8(s)) return launch_attn_tc_t<SRC, 3, 3, 2, true>(km, vm, a.q, a, sm_count, s, st);
+    if (use_tct(s)) return launch_attn_tct_t<SRC, 2, 6, 4, true>(km, vm, a.q, a, sm_count, s, st);
     if (use_fp8qs(s)) {
         if (s.rows_blk <= 16) return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);
         return launch_attn_t<SRC, 2, 2, 3, 3, true, true>(km, vm, a, sm_count, s, st);
@@ -355,6 +397,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
                 const Shape& s, cudaStream_t st, bool kv8 = false) {
     if (kv8) return launch_attn_kv8<SRC>(km, vm, a, sm_count, s, st);
     if (use_tc(s)) return launch_attn_tc<SRC>(km, vm, a.q, a, sm_count, s, st);
+    if (use_tct(s)) return launch_attn_tct_t<SRC, 2, 6, 4>(km, vm, a.q, a, sm_count, s, st);
     const int nmt = (s.rows_blk + 15) / 16;
     switch (nmt) {
         case 1:
@@ -386,6 +429,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
 
 // CTAs per SM of the variant a call with these rows will use.
 int ctas_per_sm_for(const Shape& s, bool kv8 = false) {
+    if (use_tct(s)) return 1;
     if (kv8) return use_tc8(s) ? 1 : (use_fp8qs(s) ? 3 : 2);
     if (use_tc(s)) return tc_ctas_per_sm();
     const int nmt = (s.rows_blk + 15) / 16;
