@@ -503,25 +503,53 @@ def run_gpu(args):
                 lw_, ln_ = per_label(lgw), per_label(lgn)
                 fwd_w = [a + b for a, b in zip(lw_["append_fwd"], lw_["window_fwd"])]
                 ctx_w = [a + b for a, b in zip(lw_["append_ctx"], lw_["window_ctx"])]
-                pts.append({"L": Lx,
-                            "t_fwd_draft_windowed_us": round(statistics.mean(fwd_w) * 1e3, 3),
-                            "t_fwd_draft_native_us": round(statistics.mean(ln_["full_fwd"]) * 1e3, 3),
-                            "t_ctx_draft_windowed_us": round(statistics.mean(ctx_w) * 1e3, 3),
-                            "t_ctx_draft_native_us": round(statistics.mean(ln_["full_ctx"]) * 1e3, 3),
-                            "step_windowed_us": round(max_ranks(mw) * 1e3 / Kc, 2),
-                            "step_native_us": round(max_ranks(mn) * 1e3 / Kc, 2)})
+                pt = {"L": Lx,
+                      "t_fwd_draft_windowed_us": round(statistics.mean(fwd_w) * 1e3, 3),
+                      "t_fwd_draft_native_us": round(statistics.mean(ln_["full_fwd"]) * 1e3, 3),
+                      "t_ctx_draft_windowed_us": round(statistics.mean(ctx_w) * 1e3, 3),
+                      "t_ctx_draft_native_us": round(statistics.mean(ln_["full_ctx"]) * 1e3, 3),
+                      "step_windowed_us": round(max_ranks(mw) * 1e3 / Kc, 2),
+                      "step_native_us": round(max_ranks(mn) * 1e3 / Kc, 2)}
+                if use_graph:
+                    # the same draft terms on the device alone: each term's calls captured ten
+                    # times back to back in a CUDA graph and replayed
+                    sb_ = st.b
+
+                    def fwd_win():
+                        st._append(sb_.k_fwd[0], sb_.v_fwd[0])
+                        st._window(sb_.q_fwd[0], sb_.out["fwd"], sb_.out["fwd_lse"])
+
+                    def ctx_win():
+                        st._append(sb_.k_ctx, sb_.v_ctx)
+                        st._window(sb_.q_ctx, sb_.out["ctx"], sb_.out["ctx_lse"])
+
+                    pt["t_fwd_draft_windowed_graph_us"] = round(graph_call_us([fwd_win] * 10, Kc), 3)
+                    pt["t_ctx_draft_windowed_graph_us"] = round(graph_call_us([ctx_win] * 10, Kc), 3)
+                    pt["t_fwd_draft_native_graph_us"] = round(graph_call_us(
+                        [lambda: st._full(sb_.q_fwd[0], sb_.kv_len_fwd[0], sb_.out["fwd"], sb_.out["fwd_lse"])] * 4,
+                        Kc), 3)
+                    pt["t_ctx_draft_native_graph_us"] = round(graph_call_us(
+                        [lambda: st._full(sb_.q_ctx, sb_.kv_len_ctx, sb_.out["ctx"], sb_.out["ctx_lse"])] * 4,
+                        Kc), 3)
+                    assert api.device_status() == 0
+                pts.append(pt)
                 del st
             fits = {}
             xs = [p_["L"] for p_ in pts]
-            for key in ("t_fwd_draft_windowed_us", "t_fwd_draft_native_us", "t_ctx_draft_windowed_us",
-                        "t_ctx_draft_native_us", "step_windowed_us", "step_native_us"):
+            keys = ["t_fwd_draft_windowed_us", "t_fwd_draft_native_us", "t_ctx_draft_windowed_us",
+                    "t_ctx_draft_native_us", "step_windowed_us", "step_native_us"]
+            if use_graph:
+                keys += ["t_fwd_draft_windowed_graph_us", "t_fwd_draft_native_graph_us",
+                         "t_ctx_draft_windowed_graph_us", "t_ctx_draft_native_graph_us"]
+            for key in keys:
                 m, c, r2 = acc.linear_fit(xs, [p_[key] for p_ in pts])
                 fits[key[:-3]] = {"slope_us_per_1k_tokens": round(m * 1e3, 5),
                                   "intercept_us": round(c, 3), "r2": round(r2, 5)}
             sn, sw = fits["step_native"]["slope_us_per_1k_tokens"], fits["step_windowed"]["slope_us_per_1k_tokens"]
             ctx_sweep = {"points": pts, "fits": fits, "gamma": args.gamma,
                          "step_slope_reduction_pct": round(100 * (1 - sw / sn), 2) if sn > 0 else None,
-                         "timing": "step: CUDA-graph replay; per-call terms: eager launches with events"}
+                         "timing": "step: CUDA-graph replay; per-call terms: eager launches with events, "
+                                   "and (*_graph) the same calls captured back to back in a CUDA graph"}
 
     # ---- decode loop: real acceptance from the synthetic heads, rollback, graph per step -------
     loop_res = None
