@@ -15,7 +15,6 @@
 #include "wmtp_loop.h"
 #include "attn_kernels.cuh"
 #include "attn_tc_kernels.cuh"
-#include "attn_tct_kernels.cuh"
 #include "ring_accept_kernels.cuh"
 #include "loop_kernels.cuh"
 #include "synth_kernels.cuh"
@@ -123,14 +122,9 @@ int encode_q_map(CUtensorMap* map, const void* q, int B, int n_q, int Hq, int Hk
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int min_tiles_per_cta() {
-    static int v = [] {
-        const char* e = std::getenv("WMTP_MIN_TILES");
-        int x = e ? std::atoi(e) : 2;
-        return x < 1 ? 1 : x;
-    }();
-    return v;
-}
+// Stream-K plan: a CTA takes at least this many tiles (fewer, fuller CTAs measured slower for
+// the small windowed calls, and more only lengthens the tail).
+constexpr int kMinTilesPerCta = 2;
 
 struct Shape {
     int B, n_q, Hq, Hkv, G, rows_total, rows_blk, n_rb, units;
@@ -158,17 +152,9 @@ size_t ws_total_bytes(long long slots, int rows_blk) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Launch helpers.  Kernels go out with programmatic stream serialization (PDL) unless
-// WMTP_PDL=0: each kernel lets its successor launch early and waits for its predecessor before
-// touching global memory (see pdl_wait in device_common.cuh).
-bool pdl_enabled() {
-    static bool v = [] {
-        const char* e = std::getenv("WMTP_PDL");
-        return !(e && e[0] == '0');
-    }();
-    return v;
-}
-
+// Launch helpers.  Every kernel goes out with programmatic stream serialization (PDL): it lets
+// its successor launch early and waits for its predecessor before touching global memory (see
+// pdl_wait in device_common.cuh).
 template <typename... KArgs, typename... Args>
 int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
            Args&&... args) {
@@ -181,7 +167,7 @@ int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStrea
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
         (void)cudaGetLastError();
         return WMTP_ERR_CUDA;
@@ -189,28 +175,55 @@ int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStrea
     return launched();
 }
 
-// Attention kernel variants: (key groups NKG, pipeline stages NSTAGE, CTAs per SM MINB) per
-// m-tile count NMT.  Variant 'A' is the default; WMTP_VARIANT_NMT<n>=B|C selects another (for
-// tuning sweeps).  The workspace is sized for the largest grid any variant launches.
-// Measured at 1M keys on B200 (fraction of the measured HBM copy peak; ncu shows the 1-CTA
-// layouts latency-bound with one consumer warp per sub-partition, so two independent CTA
-// pipelines per SM win once rows exceed 16):
-//   rows 16: A (4 key groups, 4 stages, 1 CTA/SM) 1.00
-//   rows 32: A (2, 2, 2 CTAs) 0.97 | (2, 4, 1) 0.81 | (1, 3, 2) 0.82
-//   rows 48: A (1, 2, 2) 0.81 | (1, 3, 2) 0.81 | (2, 4, 1) 0.70
-//   rows 64: A (1, 2, 2) 0.66 | (1, 3, 2) 0.65 | (2, 4, 1) 0.52
-constexpr int kMaxCtasPerSm = 3;
-
-char variant_for(int nmt) {
-    static char v[5] = {0, 0, 0, 0, 0};
-    if (!v[nmt]) {
-        char name[32];
-        std::snprintf(name, sizeof name, "WMTP_VARIANT_NMT%d", nmt);
-        const char* e = std::getenv(name);
-        v[nmt] = (e && (e[0] == 'B' || e[0] == 'C')) ? e[0] : 'A';
+// Sets a kernel's dynamic shared-memory limit once per device (under the library mutex, so
+// concurrent first calls from several host threads do not race on the flags).
+template <typename K>
+int set_smem_once(K kern, int bytes, bool (&done)[kMaxDevices]) {
+    int dev;
+    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return WMTP_ERR_CUDA;
+        done[dev] = true;
     }
-    return v[nmt];
+    return WMTP_OK;
 }
+
+// ---------------------------------------------------------------------------------------------
+// Kernel selection: one table, by the rows of a unit (rows_blk = min(64, n_q * G)) and the KV
+// element type.  Measured at 1M keys on B200 (fraction of the measured HBM copy peak):
+//   bf16  rows <= 16      mma.sync (1 m-tile, 4 key groups, 4 stages, 1 CTA/SM)      1.02-1.03
+//         rows 17..32     mma.sync (2, 2, 2 stages, 2 CTAs/SM)                       0.98
+//         rows 33..64     tcgen05 / TMEM (K pair slots 3, V ring 3, S buffers 2)     0.96
+//         > 64 rows       mma.sync (4, 1, 2 stages, 2 CTAs/SM) per 64-row block
+//   fp8   rows <= 16      mma.sync, Q in shared memory (1, 4, 2 stages, 3 CTAs/SM)   0.82
+//         rows 17..32     mma.sync (2, 2, 4 stages, 2 CTAs/SM)
+//         rows 33..64     tcgen05 with converter warps
+//         > 64 rows       mma.sync (4, 1, 4 stages, 2 CTAs/SM) per 64-row block
+// The 1-CTA mma.sync layouts above 16 rows were latency-bound (one consumer warp per SM
+// sub-partition); two independent CTA pipelines per SM fixed that.  The tcgen05 kernel needs
+// the whole unit in one 64-row block (its Q arrives as one TMA box of n_q x G rows).
+enum class Kern { kSplit16, kSplit32, kSplit64, kTc, kSplit16Fp8, kSplit32Fp8, kSplit64Fp8, kTcFp8 };
+
+Kern select_kernel(const Shape& s, bool kv8) {
+    const bool tc = s.rows_total <= kRowsPerBlock && s.rows_blk > 32;
+    if (tc) return kv8 ? Kern::kTcFp8 : Kern::kTc;
+    if (s.rows_blk <= 16) return kv8 ? Kern::kSplit16Fp8 : Kern::kSplit16;
+    if (s.rows_blk <= 32) return kv8 ? Kern::kSplit32Fp8 : Kern::kSplit32;
+    return kv8 ? Kern::kSplit64Fp8 : Kern::kSplit64;
+}
+
+// CTAs per SM of each kernel (the grid is sm_count times this).
+int ctas_per_sm(Kern k) {
+    switch (k) {
+        case Kern::kSplit16: return 1;
+        case Kern::kSplit16Fp8: return 3;
+        case Kern::kTc: case Kern::kTcFp8: return 1;
+        default: return 2;
+    }
+}
+constexpr int kMaxCtasPerSm = 3;
 
 template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
 int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
@@ -218,50 +231,13 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
     using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
     auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB, KV8, QS>;
     static bool attr_set[kMaxDevices] = {};
-    int dev;
-    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess)
-            return WMTP_ERR_CUDA;
-        attr_set[dev] = true;
-    }
+    int rc = set_smem_once(kern, Lay::kAlloc, attr_set);
+    if (rc != WMTP_OK) return rc;
     const int grid = sm_count * MINB;
-    int rc = launch(kern, dim3(grid), dim3((NMT * NKG + 1) * 32), Lay::kAlloc, st, km, vm, a);
+    rc = launch(kern, dim3(grid), dim3((NMT * NKG + 1) * 32), Lay::kAlloc, st, km, vm, a);
     if (rc != WMTP_OK) return rc;
     return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
-
-// Which units run on the tcgen05 kernel: by default units of 33..64 rows (at 1M keys on B200:
-// 48 rows 392 us vs 405 us for the best mma.sync layout, 64 rows 403 us vs 498 us, where the
-// legacy tensor pipe limits mma.sync); WMTP_TC=0 turns it off, WMTP_TC=all uses it for every
-// unit of at most 64 rows (tuning sweeps).
-int tc_mode() {
-    static int v = [] {
-        const char* e = std::getenv("WMTP_TC");
-        if (e && e[0] == 'a') return 2;
-        if (e && e[0] == '0') return 0;
-        return 1;
-    }();
-    return v;
-}
-
-bool use_tc(const Shape& s) {
-    if (s.rows_total > kRowsPerBlock) return false;
-    const int mode = tc_mode();
-    return mode == 2 || (mode == 1 && s.rows_blk > 32);
-}
-
-// tcgen05 kernel variants (K pair slots, V ring, S pair buffers), one CTA per SM: A = (3, 3, 2),
-// B = (2, 4, 2), C = (2, 5, 2).  WMTP_TC_VARIANT=B|C selects another (sweeps).
-char tc_variant() {
-    static char v = [] {
-        const char* e = std::getenv("WMTP_TC_VARIANT");
-        return (e && (e[0] == 'B' || e[0] == 'C')) ? e[0] : 'A';
-    }();
-    return v;
-}
-
-int tc_ctas_per_sm() { return 1; }
 
 template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
 int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
@@ -269,15 +245,10 @@ int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q
     using Lay = TcLayout<NK, NV, NSB, KV8>;
     auto kern = attn_tc_kernel<SRC, NK, NV, NSB, KV8>;
     static bool attr_set[kMaxDevices] = {};
-    int dev;
-    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess)
-            return WMTP_ERR_CUDA;
-        attr_set[dev] = true;
-    }
+    int rc = set_smem_once(kern, Lay::kAlloc, attr_set);
+    if (rc != WMTP_OK) return rc;
     CUtensorMap qm;
-    int rc = encode_q_map(&qm, q, s.B, s.n_q, s.Hq, s.Hkv);
+    rc = encode_q_map(&qm, q, s.B, s.n_q, s.Hq, s.Hkv);
     if (rc != WMTP_OK) return rc;
     const int grid = sm_count;
     rc = launch(kern, dim3(grid), dim3(tc_threads<KV8>()), Lay::kAlloc, st, km, vm, qm, a);
@@ -285,158 +256,20 @@ int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q
     return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
 }
 
-// Units of at most 32 rows on the transposed tcgen05 kernel: WMTP_TCT=1 for 17..32 rows,
-// WMTP_TCT=all for every unit of at most 32 rows (bf16 and fp8 KV).
-int tct_mode() {
-    static int v = [] {
-        const char* e = std::getenv("WMTP_TCT");
-        if (e && e[0] == 'a') return 2;
-        if (e && e[0] == '1') return 1;
-        return 0;
-    }();
-    return v;
-}
-
-bool use_tct(const Shape& s) {
-    if (s.rows_total > kTctRows) return false;
-    const int mode = tct_mode();
-    return mode == 2 || (mode == 1 && s.rows_blk > 16);
-}
-
-template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
-int launch_attn_tct_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
-                      int sm_count, const Shape& s, cudaStream_t st) {
-    using Lay = TctLayout<NK, NV, NSB, KV8>;
-    auto kern = attn_tct_kernel<SRC, NK, NV, NSB, KV8>;
-    static bool attr_set[kMaxDevices] = {};
-    int dev;
-    if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess)
-            return WMTP_ERR_CUDA;
-        attr_set[dev] = true;
-    }
-    CUtensorMap qm;
-    int rc = encode_q_map(&qm, q, s.B, s.n_q, s.Hq, s.Hkv);
-    if (rc != WMTP_OK) return rc;
-    const int grid = sm_count;
-    rc = launch(kern, dim3(grid), dim3(tct_threads<KV8>()), Lay::kAlloc, st, km, vm, qm, a);
-    if (rc != WMTP_OK) return rc;
-    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
-}
-
-template <int SRC>
-int launch_attn_tc(const CUtensorMap& km, const CUtensorMap& vm, const void* q, const AttnArgs& a,
-                   int sm_count, const Shape& s, cudaStream_t st) {
-    switch (tc_variant()) {
-        case 'B': return launch_attn_tc_t<SRC, 2, 4, 2>(km, vm, q, a, sm_count, s, st);
-        case 'C': return launch_attn_tc_t<SRC, 2, 5, 2>(km, vm, q, a, sm_count, s, st);
-        default: return launch_attn_tc_t<SRC, 3, 3, 2>(km, vm, q, a, sm_count, s, st);
-    }
-}
-
-// fp8-KV layouts per m-tile count (key groups, stages of 16 KiB, CTAs per SM), two CTAs per SM
-// throughout: widening the codes lengthens each warp's dependency chains, so the consumer warps
-// need the second CTA's warps to hide them (ncu on the one-CTA layout: 5 warps per SM, issue
-// slots 32 % busy, stalls mostly on fixed-latency dependencies).
-// fp8 units on the tcgen05 kernel (converter warps widen each tile once, in place, into fp16
-// operands): by default units of 33..64 rows, where the register-widening layouts redo the
-// work per m-tile warp (at 1M keys: 48 rows 441 vs 463 us, 64 rows 423 vs 566 us; 32 rows
-// 431 vs 345 us for the register path); WMTP_TC8=0 turns it off, WMTP_TC8=all uses it for every
-// unit of at most 64 rows.
-int tc8_mode() {
-    static int v = [] {
-        const char* e = std::getenv("WMTP_TC8");
-        if (e && e[0] == 'a') return 2;
-        if (e && e[0] == '0') return 0;
-        return 1;
-    }();
-    return v;
-}
-
-bool use_tc8(const Shape& s) {
-    if (s.rows_total > kRowsPerBlock) return false;
-    const int mode = tc8_mode();
-    return mode == 2 || (mode == 1 && s.rows_blk > 32);
-}
-
-// fp8 units with Q in shared memory and three CTAs per SM: by default units of at most 16
-// rows (the one-query draft at 1M keys: 199 vs 216 us); at 17..32 rows it measured no faster
-// (347 vs 344 us) and the two-CTA register layout stays.  WMTP_FP8QS=0 turns it off,
-// WMTP_FP8QS=all uses it up to 32 rows (sweeps).
-bool use_fp8qs(const Shape& s) {
-    static int v = [] {
-        const char* e = std::getenv("WMTP_FP8QS");
-        if (e && e[0] == 'a') return 2;
-        if (e && e[0] == '0') return 0;
-        return 1;
-    }();
-    if (use_tc8(s)) return false;
-    return (v == 1 && s.rows_blk <= 16) || (v == 2 && s.rows_blk <= 32);
-}
-
-template <int SRC>
-int launch_attn_kv8(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
-                    const Shape& s, cudaStream_t st) {
-    if (use_tc8(s)) return launch_attn_tc_t<SRC, 3, 3, 2, true>(km, vm, a.q, a, sm_count, s, st);
-    if (use_tct(s)) return launch_attn_tct_t<SRC, 2, 6, 4, true>(km, vm, a.q, a, sm_count, s, st);
-    if (use_fp8qs(s)) {
-        if (s.rows_blk <= 16) return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);
-        return launch_attn_t<SRC, 2, 2, 3, 3, true, true>(km, vm, a, sm_count, s, st);
-    }
-    switch ((s.rows_blk + 15) / 16) {
-        case 1: return launch_attn_t<SRC, 1, 4, 4, 2, true>(km, vm, a, sm_count, s, st);
-        case 2: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
-        case 3: return launch_attn_t<SRC, 3, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
-        default: return launch_attn_t<SRC, 4, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
-    }
-}
-
 template <int SRC>
 int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                 const Shape& s, cudaStream_t st, bool kv8 = false) {
-    if (kv8) return launch_attn_kv8<SRC>(km, vm, a, sm_count, s, st);
-    if (use_tc(s)) return launch_attn_tc<SRC>(km, vm, a.q, a, sm_count, s, st);
-    if (use_tct(s)) return launch_attn_tct_t<SRC, 2, 6, 4>(km, vm, a.q, a, sm_count, s, st);
-    const int nmt = (s.rows_blk + 15) / 16;
-    switch (nmt) {
-        case 1:
-            switch (variant_for(1)) {
-                case 'B': return launch_attn_t<SRC, 1, 4, 2, 2>(km, vm, a, sm_count, s, st);
-                case 'C': return launch_attn_t<SRC, 1, 2, 2, 2>(km, vm, a, sm_count, s, st);
-                default: return launch_attn_t<SRC, 1, 4, 4, 1>(km, vm, a, sm_count, s, st);
-            }
-        case 2:
-            switch (variant_for(2)) {
-                case 'B': return launch_attn_t<SRC, 2, 2, 4, 1>(km, vm, a, sm_count, s, st);
-                case 'C': return launch_attn_t<SRC, 2, 1, 3, 2>(km, vm, a, sm_count, s, st);
-                default: return launch_attn_t<SRC, 2, 2, 2, 2>(km, vm, a, sm_count, s, st);
-            }
-        case 3:
-            switch (variant_for(3)) {
-                case 'B': return launch_attn_t<SRC, 3, 1, 3, 2>(km, vm, a, sm_count, s, st);
-                case 'C': return launch_attn_t<SRC, 3, 2, 4, 1>(km, vm, a, sm_count, s, st);
-                default: return launch_attn_t<SRC, 3, 1, 2, 2>(km, vm, a, sm_count, s, st);
-            }
-        default:
-            switch (variant_for(4)) {
-                case 'B': return launch_attn_t<SRC, 4, 1, 3, 2>(km, vm, a, sm_count, s, st);
-                case 'C': return launch_attn_t<SRC, 4, 2, 4, 1>(km, vm, a, sm_count, s, st);
-                default: return launch_attn_t<SRC, 4, 1, 2, 2>(km, vm, a, sm_count, s, st);
-            }
+    switch (select_kernel(s, kv8)) {
+        case Kern::kSplit16: return launch_attn_t<SRC, 1, 4, 4, 1>(km, vm, a, sm_count, s, st);
+        case Kern::kSplit32: return launch_attn_t<SRC, 2, 2, 2, 2>(km, vm, a, sm_count, s, st);
+        case Kern::kSplit64: return launch_attn_t<SRC, 4, 1, 2, 2>(km, vm, a, sm_count, s, st);
+        case Kern::kTc: return launch_attn_tc_t<SRC, 3, 3, 2>(km, vm, a.q, a, sm_count, s, st);
+        case Kern::kSplit16Fp8: return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);
+        case Kern::kSplit32Fp8: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
+        case Kern::kSplit64Fp8: return launch_attn_t<SRC, 4, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
+        case Kern::kTcFp8: return launch_attn_tc_t<SRC, 3, 3, 2, true>(km, vm, a.q, a, sm_count, s, st);
     }
-}
-
-// CTAs per SM of the variant a call with these rows will use.
-int ctas_per_sm_for(const Shape& s, bool kv8 = false) {
-    if (use_tct(s)) return 1;
-    if (kv8) return use_tc8(s) ? 1 : (use_fp8qs(s) ? 3 : 2);
-    if (use_tc(s)) return tc_ctas_per_sm();
-    const int nmt = (s.rows_blk + 15) / 16;
-    const char v = variant_for(nmt < 4 ? nmt : 4);
-    if (nmt == 1) return v == 'A' ? 1 : 2;
-    if (nmt == 2) return v == 'B' ? 1 : 2;
-    return v == 'C' ? 1 : 2;
+    return WMTP_ERR_ARG;
 }
 
 // Common front half of the three attention calls.
@@ -452,7 +285,9 @@ int prepare(const Shape& s, const void* q, const void* out, const float* lse, vo
         return WMTP_ERR_ALIGN;
     int rc = device_info(dev);
     if (rc != WMTP_OK) return rc;
-    const long long slots = (long long)dev->sm_count * ctas_per_sm_for(s, kv8) + s.units;
+    const int grid = dev->sm_count * ctas_per_sm(select_kernel(s, kv8));
+    if (grid > kMaxParts) return WMTP_ERR_SHAPE;           // the merge's per-row weight table
+    const long long slots = (long long)grid + s.units;
     if (ws_bytes < ws_total_bytes(slots, s.rows_blk)) return WMTP_ERR_WORKSPACE;
     std::memset(a, 0, sizeof(*a));
     a->q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -466,7 +301,7 @@ int prepare(const Shape& s, const void* q, const void* out, const float* lse, vo
     a->rows_blk = s.rows_blk;
     a->scale_log2 = sm_scale * k_scale * 1.4426950408889634f;
     a->v_scale = v_scale;
-    a->min_tiles_per_cta = min_tiles_per_cta();
+    a->min_tiles_per_cta = kMinTilesPerCta;
     return WMTP_OK;
 }
 
@@ -760,8 +595,13 @@ int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k, const
                               const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D,
                               int n_sink, int window, int capacity, float sm_scale, wmtp_bf16* out,
                               float* lse, wmtp_stream_t stream) {
+    // the device check comes first, so an unsupported GPU reports WMTP_ERR_UNSUPPORTED as every
+    // other call does, before the scratch lookup
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != WMTP_OK) return rc;
     void* scratch = nullptr;
-    int rc = noalloc_scratch(&scratch);
+    rc = noalloc_scratch(&scratch);
     if (rc != WMTP_OK) return rc;
     rc = draft_attn_window(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
                            sm_scale, out, lse, scratch, WMTP_NOALLOC_SCRATCH_BYTES, stream);

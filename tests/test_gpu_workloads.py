@@ -129,9 +129,12 @@ def test_ctx128k():
     _run_workload(w, 3, 4092, _samples_factory([0, 1], w.G))
 
 
-def test_ctx1m():
+@pytest.mark.parametrize("gamma", [3, 7])
+def test_ctx1m(gamma):
+    """gamma = 3 is the benchmark's headline step (32-row verify units, 4-query context pass);
+    gamma = 7 runs the 64-row verify units on the tcgen05 kernel."""
     w = configs.CTX1M
-    _run_workload(w, 7, 4092, _samples_factory([0, 3], w.G, n_rows=4))
+    _run_workload(w, gamma, 4092, _samples_factory([0, 3], w.G, n_rows=4, seed=gamma))
 
 
 def test_batch8_ragged_tree():

@@ -3,7 +3,8 @@ their decode path (engines with a fixed memory plan, loops that cannot take cuda
 synchronisation): it must give the same result as draft_attn_window with a caller workspace.
 
 Called through the C ABI twice in a row with different shapes and inputs, so that the second
-call runs on scratch the first one left behind.  This file is collected last on purpose.
+call runs on scratch the first one left behind; each result is also checked against the fp64
+oracle.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -11,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from long_context_speculative_kv_b200 import _lib
 from synthetic import gen
 from tests.gpu_util import assert_attn_close, assert_lse_close, to_dev_bf16, to_f64
@@ -24,7 +26,8 @@ def _case(seed, B, L, Hq, Hkv, n_q, s, W):
     rng = np.random.default_rng(seed)
     C = s + W
     k_tok, v_tok = gen.kv_pair_bf16(rng, (B, L, Hkv, D))
-    q = to_dev_bf16(gen.normal_bf16(rng, (B, n_q, Hq, D)))
+    q_bits = gen.normal_bf16(rng, (B, n_q, Hq, D))
+    q = to_dev_bf16(q_bits)
     ring_k = torch.full((B, Hkv, C, D), float("nan"), dtype=torch.bfloat16, device="cuda")
     ring_v = ring_k.clone()
     rlen = torch.zeros(B, dtype=torch.int64, device="cuda")
@@ -33,7 +36,12 @@ def _case(seed, B, L, Hq, Hkv, n_q, s, W):
     rc = lib.ring_kv_append(ring_k.data_ptr(), ring_v.data_ptr(), rlen.data_ptr(), kd.data_ptr(),
                             vd.data_ptr(), B, L, Hkv, D, s, C, None)
     assert rc == 0
-    return q, ring_k, ring_v, rlen, C
+    # oracle on the linear token layout [B, Hkv, L, D]
+    ref, ref_lse = oracle.attention(q_bits, np.ascontiguousarray(k_tok.transpose(0, 2, 1, 3)),
+                                    np.ascontiguousarray(v_tok.transpose(0, 2, 1, 3)),
+                                    np.full(B, L, np.int64), oracle.MODE_WINDOW, 128 ** -0.5,
+                                    n_sink=s, window=W)
+    return q, ring_k, ring_v, rlen, C, ref, ref_lse
 
 
 def _both(q, ring_k, ring_v, rlen, Hkv, s, W, C, sc):
@@ -62,15 +70,19 @@ def _both(q, ring_k, ring_v, rlen, Hkv, s, W, C, sc):
 def test_noalloc_matches_workspace_call_twice_in_a_row():
     sc = 128 ** -0.5
     # call 1: the 1M workload's draft forward shape (B 1, GQA 32/4, one query, 4 + 4092 window)
-    q, rk, rv, rl, C = _case(11, 1, 20000, 32, 4, 1, 4, 4092)
+    q, rk, rv, rl, C, ref, ref_lse = _case(11, 1, 20000, 32, 4, 1, 4, 4092)
     (a, la), (b, lb) = _both(q, rk, rv, rl, 4, 4, 4092, C, sc)
     assert_attn_close(a, b, "noalloc call 1")
     assert_lse_close(la, lb)
+    assert_attn_close(a, ref, "noalloc call 1 vs oracle")
+    assert_lse_close(la, ref_lse)
     # call 2: a different shape on the scratch call 1 left behind (ragged batch, 4 queries)
-    q, rk, rv, rl, C = _case(12, 3, 5000, 16, 2, 4, 4, 1020)
+    q, rk, rv, rl, C, ref, ref_lse = _case(12, 3, 5000, 16, 2, 4, 4, 1020)
     (a, la), (b, lb) = _both(q, rk, rv, rl, 2, 4, 1020, C, sc)
     assert_attn_close(a, b, "noalloc call 2")
     assert_lse_close(la, lb)
+    assert_attn_close(a, ref, "noalloc call 2 vs oracle")
+    assert_lse_close(la, ref_lse)
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch():
