@@ -72,9 +72,13 @@ enum wmtp_status {
 WMTP_API const char* wmtp_status_string(int status);
 
 /* Bytes of device workspace the attention calls need for this shape on the CURRENT device
- * (split-KV partial results: one (o, lse) block per CTA per request-head it touches).  The
- * same workspace may be reused by consecutive calls on one stream; calls that may run
- * concurrently need separate workspaces.  Returns 0 for invalid shapes. */
+ * (a 256-byte control block, then split-KV partial results: one (o, lse) block per CTA per
+ * request-head it touches).  The same workspace may be reused by consecutive calls on one
+ * stream; calls that may run concurrently need separate workspaces.  Returns 0 for invalid
+ * shapes.
+ * The control block (the workspace's first 256 bytes) must be zero before the workspace's first
+ * use by draft_attn_window_append (allocate it zeroed, e.g. with cudaMemset); every call leaves
+ * it zero.  After a call whose device status reports WMTP_ERR_TIMEOUT, zero it again. */
 WMTP_API size_t wmtp_workspace_bytes(int B, int n_q, int Hq, int Hkv, int D);
 
 /* ---------------------------------------------------------------------------------------------
@@ -119,6 +123,29 @@ WMTP_API int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, cons
                       int capacity, float sm_scale,
                       wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
                       wmtp_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * draft_attn_window_append -- one draft forward in one launch: ring_kv_append of the call's new
+ * rows followed by draft_attn_window, with identical results.
+ * [verdict, pith_extraction.key_machinery]: each draft forward writes its token's draft KV and
+ * attends over the sink plus the last W tokens (t_fwd_draft in Eq. 1); [verdict,
+ * referee_report.minor_comments (App. A pseudocode)]: the KV goes to the compact ring.
+ *   Appends positions [L_old, L_old + n_new) (L_old = ring_len[b]) from k_new / v_new
+ *   [B, n_new, Hkv, D] exactly as ring_kv_append does, sets ring_len[b] = L_old + n_new, and
+ *   computes draft_attn_window with L_tot = L_old + n_new.  Usually n_new = n_q (the forward's
+ *   own tokens).  When 0 < n_new <= window the append happens inside the attention kernel (the
+ *   new rows are in the key set, so the CTA that holds a new row's slot writes it); a larger
+ *   n_new runs ring_kv_append as a separate kernel first.
+ *   ring_k, ring_v, ring_len are in/out; ws as for draft_attn_window, and its control block must
+ *   be zero (see wmtp_workspace_bytes).
+ *   Errors: those of ring_kv_append and draft_attn_window. */
+WMTP_API int draft_attn_window_append(const wmtp_bf16* q, wmtp_bf16* ring_k, wmtp_bf16* ring_v,
+                                      int64_t* ring_len, const wmtp_bf16* k_new,
+                                      const wmtp_bf16* v_new, int n_new,
+                                      int B, int n_q, int Hq, int Hkv, int D, int n_sink, int window,
+                                      int capacity, float sm_scale,
+                                      wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                                      wmtp_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * draft_attn_full -- the native MTP draft attention it replaces: causal attention over the
@@ -224,6 +251,14 @@ WMTP_API int draft_attn_window_fp8(const wmtp_bf16* q, const uint8_t* ring_k, co
                                    int capacity, float sm_scale, float k_scale, float v_scale,
                                    wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
                                    wmtp_stream_t stream);
+/* draft_attn_window_append_fp8: draft_attn_window_append on fp8 rings and fp8 new rows. */
+WMTP_API int draft_attn_window_append_fp8(const wmtp_bf16* q, uint8_t* ring_k, uint8_t* ring_v,
+                                          int64_t* ring_len, const uint8_t* k_new,
+                                          const uint8_t* v_new, int n_new,
+                                          int B, int n_q, int Hq, int Hkv, int D, int n_sink,
+                                          int window, int capacity, float sm_scale, float k_scale,
+                                          float v_scale, wmtp_bf16* out, float* lse, void* ws,
+                                          size_t ws_bytes, wmtp_stream_t stream);
 WMTP_API int draft_attn_full_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const uint8_t* v_pool,
                                  const int32_t* page_table, const int32_t* kv_len,
                                  int B, int n_q, int Hq, int Hkv, int D, int page_size, int max_pages,

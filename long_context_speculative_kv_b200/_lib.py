@@ -45,6 +45,8 @@ _SIGNATURES = {
     "wmtp_device_status": ([P], I),
     "wmtp_launch_count": ([], ctypes.c_uint64),
     "wmtp_selftest_wait_timeout": ([ctypes.c_uint64, P], I),
+    "draft_attn_window_append": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P, SZ, P], I),
+    "draft_attn_window_append_fp8": ([P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, F, F, P, P, P, SZ, P], I),
     "draft_attn_window_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P], I),
     "accept_stochastic": ([P, P, P, P, P, I, I, I, P, P, P], I),
     "ring_kv_append_fp8": ([P, P, P, P, P, I, I, I, I, I, I, P], I),

@@ -38,10 +38,11 @@ def workspace_bytes(B: int, n_q: int, Hq: int, Hkv: int, D: int = 128) -> int:
 
 
 def alloc_workspace(B: int, n_q: int, Hq: int, Hkv: int, device=None) -> torch.Tensor:
+    """A zeroed workspace (its control block must start at zero; calls leave it zero)."""
     n = workspace_bytes(B, n_q, Hq, Hkv)
     if n == 0:
         raise ValueError("invalid shape for the workspace")
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def ring_kv_append(ring_k, ring_v, ring_len, k_new, v_new, n_sink: int, stream=None) -> None:
@@ -80,6 +81,30 @@ def draft_attn_window(q, ring_k, ring_v, ring_len, n_sink: int, window: int, sm_
     check("draft_attn_window", lib().draft_attn_window(
         _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), B, n_q, Hq, Hkv, D, int(n_sink),
         int(window), C, float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def draft_attn_window_append(q, ring_k, ring_v, ring_len, k_new, v_new, n_sink: int, window: int,
+                             sm_scale: float, ws: torch.Tensor, out=None, lse=None,
+                             want_lse: bool = True, stream=None):
+    """ring_kv_append(k_new, v_new) then draft_attn_window, in one launch when the new rows fit
+    the window.  k_new, v_new [B, n_new, Hkv, 128]; ws must come from alloc_workspace (zeroed)."""
+    _want(q, torch.bfloat16, "q", 4)
+    _want(ring_k, torch.bfloat16, "ring_k", 4)
+    _want(ring_v, torch.bfloat16, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    _want(k_new, torch.bfloat16, "k_new", 4)
+    _want(v_new, torch.bfloat16, "v_new", 4)
+    B, n_q, Hq, D = q.shape
+    _, Hkv, C, _ = ring_k.shape
+    n_new = k_new.shape[1]
+    if k_new.shape != (B, n_new, Hkv, D) or v_new.shape != k_new.shape or ring_v.shape != ring_k.shape:
+        raise ValueError("draft_attn_window_append: inconsistent shapes")
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_window_append", lib().draft_attn_window_append(
+        _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), _ptr(k_new), _ptr(v_new), n_new,
+        B, n_q, Hq, Hkv, D, int(n_sink), int(window), C, float(sm_scale), _ptr(out), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream)))
     return out, lse
 
 
@@ -316,6 +341,29 @@ def draft_attn_window_fp8(q, ring_k, ring_v, ring_len, n_sink: int, window: int,
         _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), B, n_q, Hq, Hkv, D, int(n_sink),
         int(window), C, float(sm_scale), float(k_scale), float(v_scale), _ptr(out), _ptr(lse),
         _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def draft_attn_window_append_fp8(q, ring_k, ring_v, ring_len, k_new, v_new, n_sink: int, window: int,
+                                 sm_scale: float, k_scale: float, v_scale: float, ws: torch.Tensor,
+                                 out=None, lse=None, want_lse: bool = True, stream=None):
+    """draft_attn_window_append on E4M3 rings and new rows."""
+    _want(q, torch.bfloat16, "q", 4)
+    _want8(ring_k, "ring_k", 4)
+    _want8(ring_v, "ring_v", 4)
+    _want(ring_len, torch.int64, "ring_len", 1)
+    _want8(k_new, "k_new", 4)
+    _want8(v_new, "v_new", 4)
+    B, n_q, Hq, D = q.shape
+    _, Hkv, C, _ = ring_k.shape
+    n_new = k_new.shape[1]
+    if k_new.shape != (B, n_new, Hkv, D) or v_new.shape != k_new.shape or ring_v.shape != ring_k.shape:
+        raise ValueError("draft_attn_window_append_fp8: inconsistent shapes")
+    out, lse = _outs(q, out, lse, want_lse)
+    check("draft_attn_window_append_fp8", lib().draft_attn_window_append_fp8(
+        _ptr(q), _ptr(ring_k), _ptr(ring_v), _ptr(ring_len), _ptr(k_new), _ptr(v_new), n_new,
+        B, n_q, Hq, Hkv, D, int(n_sink), int(window), C, float(sm_scale), float(k_scale),
+        float(v_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return out, lse
 
 

@@ -32,14 +32,18 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in DEPS)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, ptxas_verbose: bool = False, defines=()) -> str:
+    """Compiles libwmtp.so (``defines``: extra -D options, e.g. the kernel-selection thresholds
+    of capi.cu for measurement sweeps)."""
+    if not force and not defines and not _stale():
         return LIB
-    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-o", LIB + ".tmp"] + SOURCES
+    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + [f"-D{d}" for d in defines] + \
+        ["-o", LIB + ".tmp"] + SOURCES
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv,
+                defines=[a[2:] for a in sys.argv[1:] if a.startswith("-D")]))

@@ -60,6 +60,17 @@ struct AttnArgs {
     int n_sink, window, capacity;
     // plan
     int min_tiles_per_cta;
+    // fused ring append (cluster window kernel only): positions [L_old, L_old + n_new) of each
+    // request, rows of k_new / v_new [B, n_new, Hkv, D], are written to their ring slots (and
+    // into the shared-memory tiles that hold them); the last CTA to have read ring_len advances
+    // it by n_new.  n_new = 0: no append.
+    const uint4* k_new;
+    const uint4* v_new;
+    uint4* ring_kw;              // ring K/V base (the same arrays the tensor maps read)
+    uint4* ring_vw;
+    long long* ring_len_w;       // ring_len, written once per call by the last CTA
+    unsigned int* ticket;        // workspace word, zero between calls
+    int n_new;
 };
 
 // Per-stage tile description, written by the producer before the stage's barrier completes.
@@ -70,6 +81,7 @@ struct TileMeta {
     int L_tot;      // request length (keys) including this call's n_q positions
     int flags;      // kFirst | kLast | kWhole
     int ord;        // units this CTA finished before this tile's unit (tcgen05 kernel only)
+    int slot0;      // ring slot of row 0 (ring source)
 };
 enum : int { kFirst = 1, kLast = 2, kWhole = 4 };
 
@@ -228,7 +240,38 @@ struct TileWalker {
             m.nvalid = rem < kTileKeys ? rem : kTileKeys;
             ty = r.slot0[k] + tl * kTileKeys;
             tz = b * a.Hkv + h;
+            m.slot0 = ty;
         }
+    }
+};
+
+// ---------------------------------------------------------------------------------------------
+// Cluster window mode: one unit per cluster of CL_size CTAs (grid (CL_size, units)), CTA r of
+// the cluster takes the unit's tiles [floor(r nt / CL_size), floor((r + 1) nt / CL_size)).  The
+// ring's tiles of one unit: its at most three slot ranges cut into 64-key tiles.
+struct RingUnitWalker {
+    Ranges r;
+    int b, h, rb, unit, L_tot;
+
+    __device__ __forceinline__ void describe(const AttnArgs& a, int tile, int t_begin, int t_end,
+                                             TileMeta& m, int& ty, int& tz) const {
+        int tl = tile, k = 0;
+        for (; k < r.n; ++k) {
+            const int ntk = (r.len[k] + kTileKeys - 1) / kTileKeys;
+            if (tl < ntk) break;
+            tl -= ntk;
+        }
+        if (k >= r.n) k = r.n - 1;   // unreachable: tile < tiles of the unit
+        const int rem = r.len[k] - tl * kTileKeys;
+        m.b = b; m.h = h; m.rb = rb; m.unit = unit;
+        m.L_tot = L_tot;
+        m.pos0 = r.pos0[k] + tl * kTileKeys;
+        m.nvalid = rem < kTileKeys ? rem : kTileKeys;
+        m.flags = (tile == t_begin ? kFirst : 0) | (tile == t_end - 1 ? kLast : 0);
+        m.ord = 0;
+        ty = r.slot0[k] + tl * kTileKeys;
+        tz = b * a.Hkv + h;
+        m.slot0 = ty;
     }
 };
 
@@ -273,6 +316,12 @@ struct SmemLayout {
     static constexpr int kPlanBytes = 2 * kMaxBatch * 4;            // tiles per request, length
     static constexpr int kTotal = kPlanOff + kPlanBytes;
     static constexpr int kAlloc = kTotal + 1024;                     // slack for base alignment
+    // cluster window mode: the CTA's (o, lse) partial of its unit lives in the stage space once
+    // the pipeline has drained: [NMT * 16 rows][128] fp32 normalised outputs, then the rows'
+    // base-2 LSEs
+    static constexpr int kPartOff = 0;
+    static constexpr int kPartLseOff = NMT * 16 * kD * 4;
+    static_assert(kPartLseOff + NMT * 16 * 4 <= kStagesBytes, "partial fits the stage space");
 };
 
 // Swizzled shared address of 16-byte chunk `chunk` (0..15) of key row `row` in a K/V tile
@@ -287,6 +336,57 @@ __device__ __forceinline__ uint32_t tile8_chunk_addr(uint32_t base, int row, int
 }
 
 // ---------------------------------------------------------------------------------------------
+// Cluster window mode, end of the kernel: merges the cluster's per-CTA partials of its unit
+// through distributed shared memory.  Every thread of the CTA calls it exactly once.  CTA `me`
+// takes the unit's rows me, me + size, ...; one warp per row: lane k reads rank k's LSE (ranks
+// without tiles hold no partial), then lane l sums head dims 4 l .. 4 l + 3 over the ranks with
+// one 16-byte remote load per rank.  The second cluster barrier keeps every CTA's shared memory
+// alive until its siblings have read it.
+template <int NMT, int NKG, int NSTAGE, bool KV8, bool QS>
+__device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* smem,
+                                                   const RingUnitWalker& wk, int nt, int warp,
+                                                   int lane) {
+    using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
+    constexpr int kWarps = NMT * NKG + 1;
+    cluster_sync_all();
+    const int cs = (int)gridDim.x, me = (int)blockIdx.x;
+    const int rows_u = min(kRowsPerBlock, a.rows_total - wk.rb * kRowsPerBlock);
+    const uint32_t part = smem_addr(smem + L::kPartOff);
+    const uint32_t plse = smem_addr(smem + L::kPartLseOff);
+    const bool has = lane < cs && (long long)(lane + 1) * nt / cs > (long long)lane * nt / cs;
+    for (int rr = me + warp * cs; rr < rows_u; rr += kWarps * cs) {
+        float x = -INFINITY;
+        if (has) x = ld_dsmem_f32(map_shared_rank(plse + 4u * rr, lane));
+        float mx = x;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float w = (has && mx != -INFINITY) ? exp2f(x - mx) : 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+        const uint32_t po = part + 4u * (uint32_t)(rr * kD + 4 * lane);
+        for (int k = 0; k < cs; ++k) {
+            const float wk_ = __shfl_sync(0xffffffffu, w, k);
+            if (wk_ > 0.f) {
+                const float4 v = ld_dsmem_v4(map_shared_rank(po, k));
+                acc.x += wk_ * v.x; acc.y += wk_ * v.y; acc.z += wk_ * v.z; acc.w += wk_ * v.w;
+                wsum += wk_;
+            }
+        }
+        const int R = wk.rb * kRowsPerBlock + rr;
+        const int i = R / a.G, g = R - (R / a.G) * a.G;
+        const size_t orow = ((size_t)wk.b * a.n_q + i) * a.Hq + (size_t)wk.h * a.G + g;
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        uint2 pk;
+        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(a.out + orow * kD + 4 * lane) = pk;
+        if (a.lse != nullptr && lane == 0) a.lse[orow] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
+    }
+    __syncwarp();
+    cluster_sync_all();
+}
+
+// ---------------------------------------------------------------------------------------------
 // KV8 = true: K and V are fp8 (E4M3) codes, one 128-byte row per key and head, scaled by the
 // key and value scales (the key scale folded into scale_log2).  The tiles stream at half the
 // bytes; consumers widen them to fp16 in registers (exact) and run fp16 MMAs, with Q widened to
@@ -298,12 +398,22 @@ __device__ __forceinline__ uint32_t tile8_chunk_addr(uint32_t base, int row, int
 // QS = true (fp8 only) keeps the unit's Q in shared memory as fp16 instead of in registers: each
 // A fragment is read per k-step, the kernel fits in 128 registers, and three CTAs share an SM
 // (the fp8 kernel is bound by per-warp dependency chains, so more warps per SM is what helps).
-template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
+//
+// CL = true (ring source only): the cluster window kernel.  Grid (cluster size, units), one unit
+// per cluster; each CTA streams its share of the unit's tiles, keeps its (o, lse) partial in
+// shared memory, and the cluster merges the partials through distributed shared memory (CTA r
+// merges rows r, r + size, ...), so the call is one launch with no workspace partials.  With
+// a.n_new > 0 the call also appends the request's new draft rows: the consumer warps that own a
+// new row's key slot copy it from k_new / v_new into the tile (after the TMA landed) and into
+// the ring, and the last CTA to have read ring_len advances it.
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false,
+          bool CL = false>
 __global__ void __launch_bounds__((NMT * NKG + 1) * 32, MINB)
 attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const AttnArgs a) {
     using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
     static_assert(!QS || KV8, "shared-memory Q is an fp8-KV layout");
+    static_assert(!CL || SRC == kSrcRing, "the cluster kernel reads the ring");
     constexpr int kStage = KV8 ? kStageBytes8 : kStageBytes;
     constexpr int NWC = NMT * NKG;            // consumer warps
     constexpr int KPW = kTileKeys / NKG;      // keys per consumer warp per tile
@@ -335,8 +445,48 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     pdl_wait();
 
+    __shared__ RingUnitWalker s_walk;          // cluster mode: this CTA's unit
     // ---- plan: lengths -> tiles per request -> this CTA's tile range ------------------------
-    if (warp == NWC) {
+    if (CL) {
+        if (warp == NWC && lane == 0) {
+            const int u = blockIdx.y;
+            RingUnitWalker wk;
+            wk.rb = u % a.n_rb;
+            wk.h = (u / a.n_rb) % a.Hkv;
+            wk.b = u / (a.n_rb * a.Hkv);
+            wk.unit = u;
+            const long long L_old = a.ring_len[wk.b];
+            long long Lt = L_old + a.n_new;
+            if (Lt < 0) Lt = 0;
+            if (Lt > 0x7fffffffll) Lt = 0x7fffffffll;
+            wk.L_tot = (int)Lt;
+            wk.r = ring_ranges(wk.L_tot, a.n_sink, a.window, a.capacity);
+            int nt = 0;
+            for (int k = 0; k < wk.r.n; ++k) nt += (wk.r.len[k] + kTileKeys - 1) / kTileKeys;
+            const long long cs = gridDim.x, c = blockIdx.x;
+            s_walk = wk;
+            s_range[0] = c * nt / cs;
+            s_range[1] = (c + 1) * nt / cs;
+            s_peff = nt;
+            if (a.n_new > 0) {
+                // every CTA has read its length: the last one to count in advances ring_len
+                __threadfence();
+                const unsigned int total = gridDim.x * gridDim.y;
+                if (atomicAdd(a.ticket, 1u) == total - 1u) {
+                    __threadfence();
+                    for (int b = 0; b < a.B; ++b) a.ring_len_w[b] = a.ring_len_w[b] + a.n_new;
+                    *a.ticket = 0u;
+                    __threadfence();
+                }
+            }
+            for (int s = 0; s < NSTAGE; ++s) {
+                mbar_init(&full_bar[s], 1);
+                mbar_init(&empty_bar[s], NWC);
+            }
+            mbar_init(sync_bar, NWC);
+            fence_barrier_init();
+        }
+    } else if (warp == NWC) {
         for (int b = lane; b < a.B; b += 32) {
             const int Lb = request_len<SRC>(a, b);
             plan_len[b] = Lb;
@@ -361,19 +511,22 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     __syncthreads();
     const long long t_begin = s_range[0], t_end = s_range[1];
-    if (t_begin >= t_end) return;
+    if (!CL && t_begin >= t_end) return;
 
     if (warp == NWC) {
         // =========================== producer warp =========================================
-        if (lane == 0) {
+        if (lane == 0 && t_begin < t_end) {
             const uint64_t pol = l2_evict_first_policy();
             TileWalker<SRC> walk;
-            walk.init(a, plan_tiles);
+            if (!CL) walk.init(a, plan_tiles);
             uint32_t it = 0;
             for (long long t = t_begin; t < t_end; ++t, ++it) {
                 TileMeta m;
                 int ty = 0, tz = 0;
-                walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
+                if (CL)
+                    s_walk.describe(a, (int)t, (int)t_begin, (int)t_end, m, ty, tz);
+                else
+                    walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
                 const int stage = (int)(it % NSTAGE);
                 const uint32_t phase = (it / NSTAGE) & 1u;
                 if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) break;
@@ -399,6 +552,10 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             for (uint32_t k = (issued > NSTAGE ? issued - NSTAGE : 0); k < issued; ++k) {
                 if (!mbar_wait_bounded(&empty_bar[k % NSTAGE], (k / NSTAGE) & 1u)) break;
             }
+        }
+        if (CL) {
+            __syncwarp();
+            cluster_merge_rows<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
         }
         return;
     }
@@ -444,6 +601,40 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         const uint32_t phase = (it / NSTAGE) & 1u;
         if (!mbar_wait_bounded(&full_bar[stage], phase)) { alive = false; break; }
         const TileMeta m = meta[stage];
+        bool patched = false;
+        if (CL && a.n_new > 0 && m.nvalid > 0) {
+            // fused append: the call's new positions [L_old, L_tot) that fall in this warp's keys
+            // of the tile are copied from k_new / v_new over the (stale) ring rows the TMA
+            // brought, and into the ring itself (once per unit)
+            const int L_old = m.L_tot - a.n_new;
+            const int k_hi = key0 + KPW < m.nvalid ? key0 + KPW : m.nvalid;
+            const int p_lo = max(m.pos0 + key0, L_old);
+            const int p_hi = min(m.pos0 + k_hi, m.L_tot);
+            if (p_lo < p_hi) {
+                patched = true;
+                constexpr int kChunks = KV8 ? 8 : 16;          // 16-byte pieces of a row
+                const uint32_t kb = smem_addr(smem + (size_t)stage * kStage);
+                const uint32_t vb = kb + (KV8 ? kTileBytes8 : kTileBytes);
+                for (int p = p_lo; p < p_hi; ++p) {
+                    const int row = p - m.pos0;
+                    if (lane < 2 * kChunks) {
+                        const bool isv = lane >= kChunks;
+                        const int c = isv ? lane - kChunks : lane;
+                        const size_t src_row = ((size_t)m.b * a.n_new + (p - L_old)) * a.Hkv + m.h;
+                        const uint4 val = __ldg((isv ? a.v_new : a.k_new) + src_row * kChunks + c);
+                        const uint32_t base = isv ? vb : kb;
+                        const uint32_t dst = KV8 ? tile8_chunk_addr(base, row, c) : tile_chunk_addr(base, row, c);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(dst), "r"(val.x), "r"(val.y), "r"(val.z), "r"(val.w) : "memory");
+                        if (mt == 0 && m.rb == 0) {
+                            const size_t slot = (size_t)(m.b * a.Hkv + m.h) * a.capacity + m.slot0 + row;
+                            (isv ? a.ring_vw : a.ring_kw)[slot * kChunks + c] = val;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
 
         if (m.flags & kFirst) {
             // ---- unit start: load this warp's Q rows, visibility masks, reset state -------
@@ -699,6 +890,9 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
             }
         }
+        // generic-proxy writes to the stage (the append patch) before the producer's next TMA
+        // write into it
+        if (CL && patched) fence_proxy_async();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
 
@@ -797,6 +991,10 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
                 if (!consumers_sync()) { alive = false; break; }
             }
+            if (CL && NKG == 1) {
+                // every consumer warp is past its last reads of the stage space the partial takes
+                if (!consumers_sync()) { alive = false; break; }
+            }
             if (kg == 0) {
                 const int slot = (int)blockIdx.x + m.unit;
 #pragma unroll
@@ -807,7 +1005,14 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     const float l = l_r[r];
                     const float inv = l > 0.f ? a.v_scale / l : 0.f;
                     const float lse2 = l > 0.f ? m_r[r] + __log2f(l) : -INFINITY;
-                    if (m.flags & kWhole) {
+                    if (CL) {
+                        float* po = reinterpret_cast<float*>(smem + L::kPartOff) + (size_t)rr * kD;
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            *reinterpret_cast<float2*>(po + out_dim(n, tig)) =
+                                make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+                        if (tig == 0) reinterpret_cast<float*>(smem + L::kPartLseOff)[rr] = lse2;
+                    } else if (m.flags & kWhole) {
                         const int i = R / a.G, g = R - (R / a.G) * a.G;
                         const size_t orow = ((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g;
                         uint32_t* op = reinterpret_cast<uint32_t*>(a.out + orow * kD);
@@ -826,6 +1031,10 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
             }
         }
+    }
+    if (CL) {
+        __syncwarp();
+        cluster_merge_rows<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
     }
 }
 

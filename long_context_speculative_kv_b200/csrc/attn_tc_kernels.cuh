@@ -34,10 +34,14 @@
 //                 unit's last tile combines both groups' (O, max, sum) like two split-KV partials
 //                 and writes the result, and a group starts a new unit only after that
 //                 combination (its O is then free);
-//   warps 12..15  (fp8 KV only) converters: each E4M3 tile lands in the upper half of its fp16
-//                 slot and is widened in place (two warps for K, two for V; eight warps measured
-//                 no faster); each unit's Q is widened bf16 -> fp16 in place.  The MMAs then
-//                 read fp16 operands only (P too).
+//   warps 12..15  (fp8 KV only) converters, two pairs taking alternate tiles: each E4M3 V tile
+//                 lands in the upper half of its fp16 slot and is widened in place (PV then runs
+//                 on fp16 operands, P too), and the pair that takes a unit's first tile splits the
+//                 unit's bf16 Q rows into two E4M3 terms.  K is not converted at all: QK^T runs as
+//                 kind::f8f6f4 on the E4M3 key codes as TMA lands them, against Q = 2^-k (hi + lo)
+//                 with hi = e4m3(2^k q), lo = e4m3(2^k q - hi) and one power of two 2^k per row
+//                 (bf16's 8 significant bits fit in two 4-bit E4M3 significands), and the row's
+//                 2^-k goes into its softmax scale.
 // Tensor memory: NSB S pair buffers of 128 columns, then O of group 0 and O of group 1 (128
 // columns each).  Every wait is bounded; on a timeout all roles stop, each MMA issuer waits
 // (bounded) for its own MMAs, all meet at the final barrier and warp 1 frees the tensor memory.
@@ -69,12 +73,15 @@ struct TcCols {
 // (the K-major operand of an N = 128 MMA).
 // fp8 KV: the producers land each E4M3 tile (one 128-byte x 64-key box) in the upper 64-dim half
 // of its fp16 slot, and the converter warps widen it in place (see widen_rows).
+// fp8 KV: a K pair slot holds the two tiles' E4M3 codes, [tile 0: 64 keys x 128 bytes][tile 1],
+// again 128 consecutive 128-byte rows; the Q buffer holds the unit's hi and lo E4M3 terms,
+// [64 rows x 128 bytes] each, in place of the bf16 rows the TMA brought.
 template <int NK, int NV, int NSB, bool KV8 = false>
 struct TcLayout {
     static constexpr int kPBufs = 4;                             // P buffers (one tile each)
-    static constexpr int kStage8 = KV8 ? 1 : 0;                  // (fp8: per-slot landing barriers)
+    static constexpr int kStage8 = KV8 ? 1 : 0;                  // (fp8: V landing barriers)
     static constexpr int kTileHalf = kHalfBytes;                 // 64 rows x 128 bytes
-    static constexpr int kKSlotBytes = 2 * kTileBytes;
+    static constexpr int kKSlotBytes = KV8 ? 2 * kTileBytes8 : 2 * kTileBytes;
     static constexpr int kKOff = 0;                              // NK x pair slot
     static constexpr int kVOff = kKOff + NK * kKSlotBytes;       // NV x [64 keys][128]
     static constexpr int kQOff = kVOff + NV * kTileBytes;        // 2 x [64 rows][128]
@@ -83,13 +90,16 @@ struct TcLayout {
     static constexpr int kPBytes = kHalfBytes;
     static constexpr int kBarOff = kPOff + kPBufs * kPBytes;
     // kfull[NK] kempty[NK] vfull[NV] vempty[NV] q_full[2] q_free[2] s_full[NSB] s_free[NSB]
-    // p_full[P] p_free[P] mma_done[2] merge_done; fp8: k8full[2 NK] v8full[NV] (codes landed),
-    // q_conv[2]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 2 * NSB + 2 * kPBufs + 3 +
-                                    kStage8 * (2 * NK + NV) + 2;
+    // p_full[P] p_free[P] mma_done[2] merge_done; fp8: v8full[NV] (codes landed), q_conv[2]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 2 * NSB + 2 * kPBufs + 3 + kStage8 * NV + 2;
     static constexpr int kPubOff = kBarOff + kNumBars * 8;        // per group: max[64], sum[64]
     static constexpr int kPubUnitOff = kPubOff + 2 * 2 * 64 * 4;  // per group: its last tile's unit
-    static constexpr int kKMetaOff = kPubUnitOff + 16;
+    // fp8: softmax scale of each row of the last 8 units (the unit's scale times its row's 2^-k),
+    // a ring indexed by the unit ordinal, and the V tiles' descriptions for the converters
+    static constexpr int kQScaleOff = kPubUnitOff + 16;
+    static constexpr int kQScaleRing = 8;
+    static constexpr int kVMetaOff = kQScaleOff + kStage8 * kQScaleRing * 64 * 4;
+    static constexpr int kKMetaOff = kVMetaOff + kStage8 * NV * (int)sizeof(TileMeta);
     static constexpr int kSMetaOff = kKMetaOff + 2 * NK * (int)sizeof(TileMeta);
     static constexpr int kPMetaOff = kSMetaOff + 2 * NSB * (int)sizeof(TileMeta);
     static constexpr int kPlanOff = kPMetaOff + kPBufs * (int)sizeof(TileMeta);
@@ -172,9 +182,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     uint64_t* p_free = p_full + kPB;
     uint64_t* mma_done = p_free + kPB;
     uint64_t* merge_done = mma_done + 2;
-    uint64_t* k8full = merge_done + 1;                  // fp8: [2 NK] codes of tile (slot, sub) landed
-    uint64_t* v8full = k8full + kS8 * 2 * NK;           // fp8: [NV]
-    uint64_t* q_conv = v8full + kS8 * NV;
+    uint64_t* v8full = merge_done + 1;                  // fp8: [NV] codes of a V tile landed
+    uint64_t* q_conv = v8full + kS8 * NV;               // fp8: the unit's Q split into E4M3 terms
+    float* qscale = reinterpret_cast<float*>(smem + L::kQScaleOff);     // fp8: [8 units][64 rows]
+    TileMeta* vmeta = reinterpret_cast<TileMeta*>(smem + L::kVMetaOff); // fp8: [NV]
     float* pub = reinterpret_cast<float*>(smem + L::kPubOff);           // [group][max | sum][row]
     volatile int* pub_unit = reinterpret_cast<volatile int*>(smem + L::kPubUnitOff);
     TileMeta* kmeta = reinterpret_cast<TileMeta*>(smem + L::kKMetaOff);
@@ -211,12 +222,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             const long long c = blockIdx.x;
             s_range[0] = c < peff ? cta_begin(c, T, peff) : 0;
             s_range[1] = c < peff ? cta_begin(c + 1, T, peff) : 0;
-            // K pair slot: one arrival per tile (bf16: the producer; fp8: each converter warp)
-            // (fp8: two converter warps for K and two for V, one arrival each per tile)
-            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], KV8 ? 4 : 2); mbar_init(&kempty[k], 1); }
+            // K pair slot: one arrival per tile (the producer's); V slot: the producer's (bf16) or
+            // both warps of the converter pair that widened it (fp8)
+            for (int k = 0; k < NK; ++k) { mbar_init(&kfull[k], 2); mbar_init(&kempty[k], 1); }
             for (int k = 0; k < NV; ++k) { mbar_init(&vfull[k], KV8 ? 2 : 1); mbar_init(&vempty[k], 1); }
             if (KV8) {
-                for (int k = 0; k < 2 * NK; ++k) mbar_init(&k8full[k], 1);
                 for (int k = 0; k < NV; ++k) mbar_init(&v8full[k], 1);
                 mbar_init(&q_conv[0], 2);
                 mbar_init(&q_conv[1], 2);
@@ -284,15 +294,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                     if (sub == 0u && !mbar_wait_bounded(&kempty[ks], ((pq / NK) & 1u) ^ 1u)) { alive = false; break; }
                     kmeta[2 * ks + sub] = m;
                     if (KV8) {
-                        // fp8: the codes land in the tile's upper half; the converters widen them
-                        uint64_t* lb = &k8full[2 * ks + sub];
+                        // fp8: the codes land as they are (QK^T reads E4M3 keys)
+                        uint8_t* dst8 = smem + L::kKOff + ks * L::kKSlotBytes + sub * kTileBytes8;
                         if (m.nvalid > 0) {
-                            mbar_arrive_expect_tx(lb, kTileBytes8);
-                            tma_load_3d(smem + L::kKOff + ks * L::kKSlotBytes + kTileBytes + sub * kHalfBytes,
-                                        &kmap, lb, 0, ty, tz, pol);
+                            mbar_arrive_expect_tx(&kfull[ks], kTileBytes8);
+                            tma_load_3d(dst8, &kmap, &kfull[ks], 0, ty, tz, pol);
                         } else {
-                            mbar_arrive(lb);
+                            mbar_arrive(&kfull[ks]);
                         }
+                        if (sub == 0u && t + 1 == t_end) mbar_arrive(&kfull[ks]);   // pair without tile 1
                         continue;
                     }
                     uint8_t* dst = smem + L::kKOff + ks * L::kKSlotBytes + sub * kHalfBytes;
@@ -307,6 +317,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 } else if (KV8) {
                     const uint32_t vs = it % NV;
                     if (!mbar_wait_bounded(&vempty[vs], ((it / NV) & 1u) ^ 1u)) { alive = false; break; }
+                    vmeta[vs] = m;
                     if (m.nvalid > 0) {
                         mbar_arrive_expect_tx(&v8full[vs], kTileBytes8);
                         tma_load_3d(smem + L::kVOff + vs * kTileBytes + kHalfBytes, &vmap, &v8full[vs], 0, ty, tz, pol);
@@ -336,11 +347,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     } else if (warp == 1) {
         // =========================== S issuer (QK^T) =========================================
         if (lane == 0) {
-            constexpr uint32_t kIdescS64 = KV8 ? tc::idesc_f16_f32(64, 64, false, false)
+            constexpr uint32_t kIdescS64 = KV8 ? tc::idesc_e4m3_f32(64, 64, false, false)
                                                : tc::idesc_bf16_f32(64, 64, false, false);
-            constexpr uint32_t kIdescS128 = KV8 ? tc::idesc_f16_f32(64, 128, false, false)
+            constexpr uint32_t kIdescS128 = KV8 ? tc::idesc_e4m3_f32(64, 128, false, false)
                                                 : tc::idesc_bf16_f32(64, 128, false, false);
-            uint64_t* q_ready = KV8 ? q_conv : q_full;   // fp8: Q widened to fp16 in place first
+            uint64_t* q_ready = KV8 ? q_conv : q_full;   // fp8: Q split into E4M3 terms first
             // descriptors of the ring bases; a k-step or buffer offset is added as (bytes >> 4)
             const uint64_t dK = tc::smem_desc(smem_addr(smem + L::kKOff), 16, 1024);
             const uint64_t dQ = tc::smem_desc(smem_addr(smem + L::kQOff), 16, 1024);
@@ -368,7 +379,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 tc::fence_after_sync();
                 const uint32_t kslot = ks * (uint32_t)L::kKSlotBytes;
                 const bool paired = has1 && mt[0].nvalid > 0 && mt[1].nvalid > 0 && mt[0].unit == mt[1].unit;
-                if (paired) {
+                if (KV8) {
+                    // E4M3: k-step j covers dims 32 j .. 32 j + 31 (32 bytes of every row); the hi
+                    // and lo terms of Q accumulate into the same scores
+                    if (paired) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t qoff = qb[0] * (uint32_t)L::kQBytes + (uint32_t)((j >> 2) * kHalfBytes + (j & 3) * 32);
+                            const uint32_t koff = kslot + (uint32_t)((j & 3) * 32);
+                            tc::mma_f8_ss(tmem + sb * 128u, dQ + (qoff >> 4), dK + (koff >> 4), kIdescS128, j > 0);
+                        }
+                    } else {
+                        for (uint32_t sub = 0; sub < (has1 ? 2u : 1u); ++sub) {
+                            if (mt[sub].nvalid <= 0) continue;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const uint32_t qoff = qb[sub] * (uint32_t)L::kQBytes +
+                                                      (uint32_t)((j >> 2) * kHalfBytes + (j & 3) * 32);
+                                const uint32_t koff = kslot + sub * (uint32_t)kTileBytes8 + (uint32_t)((j & 3) * 32);
+                                tc::mma_f8_ss(tmem + sb * 128u + 64u * sub, dQ + (qoff >> 4), dK + (koff >> 4),
+                                              kIdescS64, j > 0);
+                            }
+                        }
+                    }
+                } else if (paired) {
                     // one N = 128 MMA per k-step: keys of both tiles are consecutive rows
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -434,55 +468,97 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         }
     } else if (KV8 && warp >= 12) {
         // =========================== converters (fp8 KV) =====================================
-        // warps 12-13 widen each K tile in its pair slot (and each unit's Q rows to fp16 in
-        // place), warps 14-15 each V tile in its V slot; thread r owns key row r.  The MMAs read
-        // only fp16 operands.
-        const bool conv_k = warp < 14;
-        const int r = threadIdx.x - (conv_k ? 384 : 448);          // 0 .. 63
-        uint32_t uq = 0;
-        for (uint32_t t = 0; t < n; ++t) {
-            if (conv_k) {
-                const uint32_t pq = t >> 1, sub = t & 1u, ks = pq % NK;
-                if (!mbar_wait_bounded(&k8full[2 * ks + sub], (pq / NK) & 1u)) break;
-                const TileMeta m = kmeta[2 * ks + sub];
-                if (m.flags & kFirst) {
-                    const uint32_t qb = uq & 1u;
-                    if (!mbar_wait_bounded(&q_full[qb], (uq >> 1) & 1u)) break;
-                    const uint32_t qa = smem_addr(smem + L::kQOff + qb * L::kQBytes);
-                    for (int i = r; i < L::kQBytes / 16; i += 64) {
-                        uint32_t v0, v1, v2, v3;
+        // Pair 0 (warps 12-13) takes the even tiles, pair 1 (warps 14-15) the odd ones.  Thread r
+        // of a pair owns key row r of its V tiles (widened to fp16 in place) and, at a unit's
+        // first tile, query row r of the unit (split in place into the E4M3 hi and lo terms).
+        const uint32_t pair = (uint32_t)(warp - 12) >> 1;
+        const int r = threadIdx.x - 384 - 64 * (int)pair;            // 0 .. 63
+        for (uint32_t t = pair; t < n; t += 2) {
+            const uint32_t vs = t % NV;
+            if (!mbar_wait_bounded(&v8full[vs], (t / NV) & 1u)) break;
+            const TileMeta m = vmeta[vs];
+            if (m.flags & kFirst) {
+                const uint32_t u = (uint32_t)m.ord, qb = u & 1u;
+                if (!mbar_wait_bounded(&q_full[qb], (u >> 1) & 1u)) break;
+                const uint32_t row = smem_addr(smem + L::kQOff + qb * L::kQBytes) + (uint32_t)(r * 128);
+                const bool live = r < a.rows_total - m.rb * kRowsPerBlock;
+                // chunk c of the bf16 boxes (box c / 8): dims 8 c .. 8 c + 7 of the row
+                auto bchunk = [&](int c) -> uint32_t {
+                    return row + (uint32_t)((c >> 3) * kHalfBytes) + (uint32_t)(((c & 7) ^ (r & 7)) << 4);
+                };
+                float amax = 0.f;
+                if (live) {
+#pragma unroll 4
+                    for (int c = 0; c < 16; ++c) {
+                        uint32_t w4[4];
                         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3) : "r"(qa + 16u * i));
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                                     :: "r"(qa + 16u * i), "r"(bf16x2_to_f16x2(v0)), "r"(bf16x2_to_f16x2(v1)),
-                                        "r"(bf16x2_to_f16x2(v2)), "r"(bf16x2_to_f16x2(v3))
-                                     : "memory");
+                                     : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3]) : "r"(bchunk(c)) : "memory");
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[k] << 16)),
+                                                     fabsf(__uint_as_float(w4[k] & 0xffff0000u))));
                     }
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&q_conv[qb]);
-                    ++uq;
                 }
-                if (m.nvalid > 0) {
-                    const uint32_t base = smem_addr(smem + L::kKOff + ks * L::kKSlotBytes + sub * kHalfBytes);
-                    widen_rows(base + kTileBytes, base, m.nvalid, r);
+                // 2^k q < 2^8 for the row's largest |q| (E4M3 reaches 448); the row's scores come
+                // out 2^k too large, so its softmax scale carries 2^-k
+                int e = 0;
+                if (amax > 0.f) (void)frexpf(amax, &e);
+                const int k2 = 8 - e;
+                const float up = ldexpf(1.f, k2);
+                qscale[(u % L::kQScaleRing) * 64 + r] = ldexpf(a.scale_log2, -k2);
+                // output chunk c holds the codes of dims 16 c .. 16 c + 15 (lowest dim in the lowest
+                // byte): hi in chunk c of box 0's space, lo in chunk c of box 1's space.  Writing hi
+                // chunk c clobbers bf16 dims 8 c .. of box 0, which output chunks <= c have read
+                // already; the lo chunks would clobber box 1 dims still unread, so they are held
+                // in registers and written last.
+                uint32_t lo[8][4];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t w8[8];
+                    if (live) {
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w8[0]), "=r"(w8[1]), "=r"(w8[2]), "=r"(w8[3]) : "r"(bchunk(2 * c)) : "memory");
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w8[4]), "=r"(w8[5]), "=r"(w8[6]), "=r"(w8[7]) : "r"(bchunk(2 * c + 1)) : "memory");
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) w8[k] = 0u;
+                    }
+                    uint32_t hi4[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t wa = w8[2 * k], wb = w8[2 * k + 1];
+                        const float x0 = __uint_as_float(wa << 16) * up;
+                        const float x1 = __uint_as_float(wa & 0xffff0000u) * up;
+                        const float x2 = __uint_as_float(wb << 16) * up;
+                        const float x3 = __uint_as_float(wb & 0xffff0000u) * up;
+                        hi4[k] = f32x2_to_e4m3x2(x0, x1) | (f32x2_to_e4m3x2(x2, x3) << 16);
+                        uint32_t h01, h23;
+                        e4m3x4_to_f16x2x2(hi4[k], h01, h23);
+                        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                        lo[c][k] = f32x2_to_e4m3x2(x0 - v01.x, x1 - v01.y) |
+                                   (f32x2_to_e4m3x2(x2 - v23.x, x3 - v23.y) << 16);
+                    }
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                 :: "r"(row + (uint32_t)((c ^ (r & 7)) << 4)), "r"(hi4[0]), "r"(hi4[1]),
+                                    "r"(hi4[2]), "r"(hi4[3]) : "memory");
                 }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                 :: "r"(row + (uint32_t)kHalfBytes + (uint32_t)((c ^ (r & 7)) << 4)),
+                                    "r"(lo[c][0]), "r"(lo[c][1]), "r"(lo[c][2]), "r"(lo[c][3]) : "memory");
                 fence_proxy_async();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&kfull[ks]);
-                    if (sub == 0u && t + 1 == n) mbar_arrive(&kfull[ks]);   // pair without tile 1
-                }
-            } else {
-                const uint32_t vs = t % NV;
-                if (!mbar_wait_bounded(&v8full[vs], (t / NV) & 1u)) break;
-                // rows past the valid keys come out as zeros (codes there may be anything)
-                const uint32_t base = smem_addr(smem + L::kVOff + vs * kTileBytes);
-                widen_rows(base + kHalfBytes, base, kTileKeys, r);
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&vfull[vs]);
+                if (lane == 0) mbar_arrive(&q_conv[qb]);
             }
+            // rows past the valid keys come out as zeros (codes there may be anything)
+            const uint32_t base = smem_addr(smem + L::kVOff + vs * kTileBytes);
+            widen_rows(base + kHalfBytes, base, kTileKeys, r);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&vfull[vs]);
         }
     } else {
         // =========================== softmax warps (two groups) ==============================
@@ -499,6 +575,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         const float* pub_m_oth = pub + (2 * (grp ^ 1u)) * 64;
         const float* pub_l_oth = pub + (2 * (grp ^ 1u) + 1) * 64;
         float m_used = -INFINITY, l_part = 0.f;
+        float rs = a.scale_log2;                         // this row's score scale (log2 units)
         unsigned long long vis = 0ull;
         bool row_ok = false;
         int Lpre = 0, my_unit = -1;
@@ -524,6 +601,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 vis = row_ok ? step_visibility(a, m.b, R / a.G) : 0ull;
                 m_used = -INFINITY;
                 l_part = 0.f;
+                // fp8: the row's Q carries 2^k (written before the unit's first QK^T was issued,
+                // so before these scores completed)
+                if (KV8) rs = qscale[((uint32_t)m.ord % L::kQScaleRing) * 64 + row];
             }
             // ---- this thread's 32 scores from tensor memory ---------------------------------
             __syncwarp();
@@ -564,7 +644,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(fmaxf(x[j], x[j + 8]), fmaxf(x[j + 16], x[j + 24]));
             float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * a.scale_log2;
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * rs;
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + kRescaleThreshold || (m_used == -INFINITY && mx != -INFINITY)) {
@@ -580,8 +660,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float p0 = fast_exp2(fmaf(x[2 * j], a.scale_log2, -m_sub));
-                const float p1 = fast_exp2(fmaf(x[2 * j + 1], a.scale_log2, -m_sub));
+                const float p0 = fast_exp2(fmaf(x[2 * j], rs, -m_sub));
+                const float p1 = fast_exp2(fmaf(x[2 * j + 1], rs, -m_sub));
                 if (KV8) {
                     // fp16 weights for the fp16 V; the row sum over the same rounded weights
                     pk[j] = pack_f16x2(p0, p1);

@@ -143,12 +143,14 @@ int check_shape(int B, int n_q, int Hq, int Hkv, int D, Shape* s) {
     return WMTP_OK;
 }
 
-// Workspace: [slots][rows_blk][128] fp32 partial outputs, then [slots][rows_blk] fp32 partial
-// LSEs (slot = CTA + unit; rows_blk = rows per unit).
+// Workspace: a 256-byte control block (word 0: the fused append's ticket, zero between calls),
+// then [slots][rows_blk][128] fp32 partial outputs, then [slots][rows_blk] fp32 partial LSEs
+// (slot = CTA + unit; rows_blk = rows per unit).
+constexpr size_t kWsControl = 256;
 size_t ws_o_bytes(long long slots, int rows_blk) { return (size_t)slots * rows_blk * kD * sizeof(float); }
 size_t ws_total_bytes(long long slots, int rows_blk) {
     size_t a = (ws_o_bytes(slots, rows_blk) + 255) & ~size_t(255);
-    return a + (size_t)slots * rows_blk * sizeof(float);
+    return kWsControl + a + (size_t)slots * rows_blk * sizeof(float);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -168,6 +170,31 @@ int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStrea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return WMTP_ERR_CUDA;
+    }
+    return launched();
+}
+
+// The same with a cluster of `cs` CTAs along x.
+template <typename... KArgs, typename... Args>
+int launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   int cs, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cs;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
         (void)cudaGetLastError();
         return WMTP_ERR_CUDA;
@@ -204,10 +231,18 @@ int set_smem_once(K kern, int bytes, bool (&done)[kMaxDevices]) {
 // The 1-CTA mma.sync layouts above 16 rows were latency-bound (one consumer warp per SM
 // sub-partition); two independent CTA pipelines per SM fixed that.  The tcgen05 kernel needs
 // the whole unit in one 64-row block (its Q arrives as one TMA box of n_q x G rows).
+// Build-time option for measurement sweeps: the smallest unit (in rows) the tcgen05 kernel takes,
+// bf16 and fp8 KV (default 33 for both).
+#ifndef WMTP_TC_MIN_ROWS
+#define WMTP_TC_MIN_ROWS 33
+#endif
+#ifndef WMTP_TC8_MIN_ROWS
+#define WMTP_TC8_MIN_ROWS 33
+#endif
 enum class Kern { kSplit16, kSplit32, kSplit64, kTc, kSplit16Fp8, kSplit32Fp8, kSplit64Fp8, kTcFp8 };
 
 Kern select_kernel(const Shape& s, bool kv8) {
-    const bool tc = s.rows_total <= kRowsPerBlock && s.rows_blk > 32;
+    const bool tc = s.rows_total <= kRowsPerBlock && s.rows_blk >= (kv8 ? WMTP_TC8_MIN_ROWS : WMTP_TC_MIN_ROWS);
     if (tc) return kv8 ? Kern::kTcFp8 : Kern::kTc;
     if (s.rows_blk <= 16) return kv8 ? Kern::kSplit16Fp8 : Kern::kSplit16;
     if (s.rows_blk <= 32) return kv8 ? Kern::kSplit32Fp8 : Kern::kSplit32;
@@ -272,6 +307,86 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
     return WMTP_ERR_ARG;
 }
 
+// ---------------------------------------------------------------------------------------------
+// The windowed draft call: the cluster window kernel, one unit per cluster.  The cluster size is
+// the largest of 16, 8, 4, 2 that leaves every CTA at least two tiles of the longest possible
+// window and lets all units' clusters be resident at once (the occupancy query counts the
+// clusters the GPU can hold with this kernel's shared memory); else 1 (one CTA per unit, no
+// merge).  Queried once per device, kernel and size.
+template <typename K>
+int cluster_capacity(K kern, int smem, int threads, int cs, int (&cache)[kMaxDevices][5],
+                     bool (&init)[kMaxDevices][5]) {
+    int dev;
+    if (current_device(&dev) != WMTP_OK) return 0;
+    const int k = cs == 16 ? 4 : cs == 8 ? 3 : cs == 4 ? 2 : cs == 2 ? 1 : 0;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!init[dev][k]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cs, 1, 1);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = 0;
+        }
+        cache[dev][k] = n;
+        init[dev][k] = true;
+    }
+    return cache[dev][k];
+}
+
+template <int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
+int launch_window_cluster_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
+                            const Shape& s, int max_tiles, cudaStream_t st) {
+    using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
+    auto kern = attn_split_kernel<kSrcRing, NMT, NKG, NSTAGE, MINB, KV8, QS, true>;
+    constexpr int kThreads = (NMT * NKG + 1) * 32;
+    static bool attr_set[kMaxDevices] = {};
+    static int cap[kMaxDevices][5];
+    static bool cap_init[kMaxDevices][5] = {};
+    {
+        int dev;
+        if (current_device(&dev) != WMTP_OK) return WMTP_ERR_CUDA;
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc) != cudaSuccess ||
+                cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+                return WMTP_ERR_CUDA;
+            attr_set[dev] = true;
+        }
+    }
+    int cs = 1;
+    for (int c = 16; c >= 2; c >>= 1) {
+        if (2 * c > max_tiles) continue;
+        const int n = cluster_capacity(kern, Lay::kAlloc, kThreads, c, cap, cap_init);
+        if (n > 0 && s.units <= n) { cs = c; break; }
+    }
+    return launch_cluster(kern, dim3(cs, s.units), dim3(kThreads), Lay::kAlloc, st, cs, km, vm, a);
+}
+
+int launch_window_cluster(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
+                          const Shape& s, int max_tiles, cudaStream_t st, bool kv8) {
+    switch (select_kernel(s, kv8)) {
+        case Kern::kSplit16: return launch_window_cluster_t<1, 4, 4, 1>(km, vm, a, s, max_tiles, st);
+        case Kern::kSplit32: return launch_window_cluster_t<2, 2, 2, 2>(km, vm, a, s, max_tiles, st);
+        case Kern::kSplit64: case Kern::kTc:
+            return launch_window_cluster_t<4, 1, 2, 2>(km, vm, a, s, max_tiles, st);
+        case Kern::kSplit16Fp8: return launch_window_cluster_t<1, 4, 2, 3, true, true>(km, vm, a, s, max_tiles, st);
+        case Kern::kSplit32Fp8: return launch_window_cluster_t<2, 2, 4, 2, true>(km, vm, a, s, max_tiles, st);
+        case Kern::kSplit64Fp8: case Kern::kTcFp8:
+            return launch_window_cluster_t<4, 1, 4, 2, true>(km, vm, a, s, max_tiles, st);
+    }
+    return WMTP_ERR_ARG;
+}
+
 // Common front half of the three attention calls.
 int prepare(const Shape& s, const void* q, const void* out, const float* lse, void* ws,
             size_t ws_bytes, float sm_scale, DeviceInfo* dev, AttnArgs* a, bool kv8 = false,
@@ -293,8 +408,10 @@ int prepare(const Shape& s, const void* q, const void* out, const float* lse, vo
     a->q = reinterpret_cast<const __nv_bfloat16*>(q);
     a->out = reinterpret_cast<__nv_bfloat16*>(const_cast<void*>(out));
     a->lse = const_cast<float*>(lse);
-    a->ws_o = reinterpret_cast<float*>(ws);
-    a->ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+    a->ticket = reinterpret_cast<unsigned int*>(wsb);
+    a->ws_o = reinterpret_cast<float*>(wsb + kWsControl);
+    a->ws_lse = reinterpret_cast<float*>(wsb + kWsControl +
                                          ((ws_o_bytes(slots, s.rows_blk) + 255) & ~size_t(255)));
     a->B = s.B; a->n_q = s.n_q; a->Hq = s.Hq; a->Hkv = s.Hkv; a->G = s.G; a->n_rb = s.n_rb;
     a->rows_total = s.rows_total;
@@ -455,10 +572,15 @@ int ring_append_call(void* ring_k, void* ring_v, int64_t* ring_len, const void* 
                   reinterpret_cast<long long*>(ring_len), B, n_new);
 }
 
-int window_call(const wmtp_bf16* q, const void* ring_k, const void* ring_v, const int64_t* ring_len,
+// The windowed draft call, optionally with the ring append of the call's new rows fused in
+// (n_new > 0: positions [ring_len[b], ring_len[b] + n_new) get the rows of k_new / v_new and
+// ring_len advances, as ring_kv_append would).  stream_k: the stream-K kernel with workspace
+// partials and the LSE merge kernel instead of the cluster kernel (the no-alloc entry point).
+int window_call(const wmtp_bf16* q, void* ring_k, void* ring_v, int64_t* ring_len,
+                const void* k_new, const void* v_new, int n_new,
                 int B, int n_q, int Hq, int Hkv, int D, int n_sink, int window, int capacity,
                 float sm_scale, wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes,
-                wmtp_stream_t stream, bool kv8, float k_scale, float v_scale) {
+                wmtp_stream_t stream, bool kv8, float k_scale, float v_scale, bool stream_k = false) {
     Shape s;
     int rc = check_shape(B, n_q, Hq, Hkv, D, &s);
     if (rc != WMTP_OK) return rc;
@@ -466,18 +588,46 @@ int window_call(const wmtp_bf16* q, const void* ring_k, const void* ring_v, cons
     if (n_sink < 0 || window < 0 || capacity <= n_sink || window > capacity - n_sink) return WMTP_ERR_ARG;
     if ((long long)B * Hkv > 0x7fffffffll) return WMTP_ERR_SHAPE;
     if (!aligned(ring_k, 16) || !aligned(ring_v, 16) || !aligned(ring_len, 8)) return WMTP_ERR_ALIGN;
+    if (n_new < 0) return WMTP_ERR_ARG;
+    if (n_new > 0) {
+        if (k_new == nullptr || v_new == nullptr) return WMTP_ERR_ARG;
+        if (!aligned(k_new, 16) || !aligned(v_new, 16)) return WMTP_ERR_ALIGN;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the fused append covers new rows that all fall in the call's key set (n_new <= window);
+    // otherwise the append runs as its own kernel first
+    const bool fused = n_new > 0 && n_new <= window && !stream_k && s.units <= 65535;
     DeviceInfo dev;
     AttnArgs a;
     rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a, kv8, k_scale, v_scale);
     if (rc != WMTP_OK) return rc;
+    if (n_new > 0 && !fused) {
+        rc = kv8 ? ring_append_call<8>(ring_k, ring_v, ring_len, k_new, v_new, B, n_new, Hkv, D, n_sink,
+                                       capacity, stream)
+                 : ring_append_call<16>(ring_k, ring_v, ring_len, k_new, v_new, B, n_new, Hkv, D, n_sink,
+                                        capacity, stream);
+        if (rc != WMTP_OK) return rc;
+    }
     a.ring_len = reinterpret_cast<const long long*>(ring_len);
+    a.ring_len_w = reinterpret_cast<long long*>(ring_len);
     a.n_sink = n_sink;
     a.window = window;
     a.capacity = capacity;
+    if (fused) {
+        a.k_new = reinterpret_cast<const uint4*>(k_new);
+        a.v_new = reinterpret_cast<const uint4*>(v_new);
+        a.ring_kw = reinterpret_cast<uint4*>(ring_k);
+        a.ring_vw = reinterpret_cast<uint4*>(ring_v);
+        a.n_new = n_new;
+    }
     CUtensorMap km, vm;
     if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
     if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
-    return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, reinterpret_cast<cudaStream_t>(stream), kv8);
+    if (stream_k || s.units > 65535)
+        return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, st, kv8);
+    // tiles of the longest key set: the sink's, the window's, one more where the window wraps
+    const int max_tiles = (n_sink + kTileKeys - 1) / kTileKeys + (window + kTileKeys - 1) / kTileKeys + 1;
+    return launch_window_cluster(km, vm, a, s, max_tiles, st, kv8);
 }
 
 }  // namespace
@@ -503,16 +653,35 @@ int draft_attn_window(const wmtp_bf16* q, const wmtp_bf16* ring_k, const wmtp_bf
                       const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D, int n_sink,
                       int window, int capacity, float sm_scale, wmtp_bf16* out, float* lse, void* ws,
                       size_t ws_bytes, wmtp_stream_t stream) {
-    return window_call(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
-                       sm_scale, out, lse, ws, ws_bytes, stream, false, 1.f, 1.f);
+    return window_call(q, const_cast<wmtp_bf16*>(ring_k), const_cast<wmtp_bf16*>(ring_v),
+                       const_cast<int64_t*>(ring_len), nullptr, nullptr, 0, B, n_q, Hq, Hkv, D, n_sink,
+                       window, capacity, sm_scale, out, lse, ws, ws_bytes, stream, false, 1.f, 1.f);
+}
+
+int draft_attn_window_append(const wmtp_bf16* q, wmtp_bf16* ring_k, wmtp_bf16* ring_v, int64_t* ring_len,
+                             const wmtp_bf16* k_new, const wmtp_bf16* v_new, int n_new, int B, int n_q,
+                             int Hq, int Hkv, int D, int n_sink, int window, int capacity, float sm_scale,
+                             wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes, wmtp_stream_t stream) {
+    return window_call(q, ring_k, ring_v, ring_len, k_new, v_new, n_new, B, n_q, Hq, Hkv, D, n_sink,
+                       window, capacity, sm_scale, out, lse, ws, ws_bytes, stream, false, 1.f, 1.f);
+}
+
+int draft_attn_window_append_fp8(const wmtp_bf16* q, uint8_t* ring_k, uint8_t* ring_v, int64_t* ring_len,
+                                 const uint8_t* k_new, const uint8_t* v_new, int n_new, int B, int n_q,
+                                 int Hq, int Hkv, int D, int n_sink, int window, int capacity,
+                                 float sm_scale, float k_scale, float v_scale, wmtp_bf16* out, float* lse,
+                                 void* ws, size_t ws_bytes, wmtp_stream_t stream) {
+    return window_call(q, ring_k, ring_v, ring_len, k_new, v_new, n_new, B, n_q, Hq, Hkv, D, n_sink,
+                       window, capacity, sm_scale, out, lse, ws, ws_bytes, stream, true, k_scale, v_scale);
 }
 
 int draft_attn_window_fp8(const wmtp_bf16* q, const uint8_t* ring_k, const uint8_t* ring_v,
                           const int64_t* ring_len, int B, int n_q, int Hq, int Hkv, int D, int n_sink,
                           int window, int capacity, float sm_scale, float k_scale, float v_scale,
                           wmtp_bf16* out, float* lse, void* ws, size_t ws_bytes, wmtp_stream_t stream) {
-    return window_call(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
-                       sm_scale, out, lse, ws, ws_bytes, stream, true, k_scale, v_scale);
+    return window_call(q, const_cast<uint8_t*>(ring_k), const_cast<uint8_t*>(ring_v),
+                       const_cast<int64_t*>(ring_len), nullptr, nullptr, 0, B, n_q, Hq, Hkv, D, n_sink,
+                       window, capacity, sm_scale, out, lse, ws, ws_bytes, stream, true, k_scale, v_scale);
 }
 
 int draft_attn_full_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const uint8_t* v_pool,
@@ -603,8 +772,10 @@ int draft_attn_window_noalloc(const wmtp_bf16* q, const wmtp_bf16* ring_k, const
     void* scratch = nullptr;
     rc = noalloc_scratch(&scratch);
     if (rc != WMTP_OK) return rc;
-    rc = draft_attn_window(q, ring_k, ring_v, ring_len, B, n_q, Hq, Hkv, D, n_sink, window, capacity,
-                           sm_scale, out, lse, scratch, WMTP_NOALLOC_SCRATCH_BYTES, stream);
+    rc = window_call(q, const_cast<wmtp_bf16*>(ring_k), const_cast<wmtp_bf16*>(ring_v),
+                     const_cast<int64_t*>(ring_len), nullptr, nullptr, 0, B, n_q, Hq, Hkv, D, n_sink, window,
+                     capacity, sm_scale, out, lse, scratch, WMTP_NOALLOC_SCRATCH_BYTES, stream, false, 1.f,
+                     1.f, /*stream_k=*/true);
     return rc == WMTP_ERR_WORKSPACE ? WMTP_ERR_SCRATCH_LIMIT : rc;
 }
 

@@ -122,6 +122,35 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------------------
+// Thread-block clusters: the hardware cluster barrier (every thread of every CTA of the cluster
+// arrives; release / acquire order shared-memory writes before it with reads after it) and
+// loads from another CTA's shared memory (distributed shared memory; no TMA, no multicast).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------------------------------------
 // ldmatrix / mma.sync (bf16 in, fp32 accumulate).
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -174,6 +203,14 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, 
         "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
         "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
         : "=r"(lo), "=r"(hi) : "r"(codes));
+}
+
+// Two fp32 values -> two E4M3 codes (round to nearest even, saturating at +-448): `lo` in the
+// lower byte, `hi` in the upper.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return (uint32_t)d;
 }
 
 // bf16x2 -> fp16x2 through fp32 (exact for values fp16 represents).

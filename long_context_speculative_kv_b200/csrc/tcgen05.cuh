@@ -1,6 +1,7 @@
 // tcgen05.cuh -- 5th-generation tensor core (tcgen05) helpers for sm_100a: tensor-memory
 // allocation, MMA issue and completion, tensor-memory loads/stores, and the shared-memory and
-// instruction descriptors of kind::f16 (bf16 inputs, fp32 accumulators).
+// instruction descriptors of kind::f16 (bf16 / fp16 inputs) and kind::f8f6f4 (E4M3 inputs), both
+// with fp32 accumulators.
 #pragma once
 
 #include <stdint.h>
@@ -37,6 +38,18 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The same for 8-bit operands (kind::f8f6f4; here E4M3 x E4M3 -> fp32): K = 32 per instruction,
+// i.e. 32 bytes of each operand row, as kind::f16's K = 16.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -121,6 +134,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t smem_byte_addr, uint32_t 
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
            ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// kind::f8f6f4 with E4M3 A and B (format code 0) and an fp32 accumulator: the same fields.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 // The same with fp16 A and B (format code 0).
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {

@@ -10,7 +10,8 @@ pith_extraction.key_machinery, Eq. 1: t_step = t_verify + t_ctx_draft + gamma * 
     step's draft-forward rows), then one draft attention call with n_q = gamma + 1 (the worst
     case of the pages' accounting; queries before the newly committed ones re-read older
     positions);
-  * gamma draft forwards: ring_kv_append of one row, draft attention with n_q = 1;
+  * gamma draft forwards: ring append of one row and draft attention with n_q = 1, one library
+    call (draft_attn_window_append);
   * proposals: the synthetic draft head (tokens [B, gamma + 1], node 0 = last committed token);
   * verify: one verify_attn per target attention layer over T - 1 + gamma + 1 keys;
   * the synthetic target head's logits for the gamma + 1 nodes, accept_greedy, spec_commit.
@@ -89,7 +90,7 @@ class DecodeLoop:
         if bufs.ws is None:
             Hq = bufs.q_verify.shape[3]
             Hkv = bufs.k_pools[0].shape[1]
-            bufs.ws = torch.empty(max(api.workspace_bytes(B, n_q, Hq, Hkv), api.workspace_bytes(B, 1, Hq, Hkv)),
+            bufs.ws = torch.zeros(max(api.workspace_bytes(B, n_q, Hq, Hkv), api.workspace_bytes(B, 1, Hq, Hkv)),
                                   dtype=torch.uint8, device=dev)
         if bufs.ring_k is not None and bufs.ring_k.shape[2] < bufs.n_sink + bufs.window + gamma:
             raise ValueError("ring capacity must be >= n_sink + window + gamma for the rollback")
@@ -103,11 +104,10 @@ class DecodeLoop:
         api.draft_attn_window(b.q_ctx, b.ring_k, b.ring_v, b.ring_len, b.n_sink, b.window, b.sm_scale, b.ws,
                               out=b.out["ctx"], lse=b.out["ctx_lse"])
         for j in range(self.gamma):
-            if log: log.mark("append_fwd")
-            api.ring_kv_append(b.ring_k, b.ring_v, b.ring_len, b.k_fwd[j], b.v_fwd[j], b.n_sink)
             if log: log.mark("window_fwd")
-            api.draft_attn_window(b.q_fwd[j], b.ring_k, b.ring_v, b.ring_len, b.n_sink, b.window,
-                                  b.sm_scale, b.ws, out=b.out["fwd"], lse=b.out["fwd_lse"])
+            api.draft_attn_window_append(b.q_fwd[j], b.ring_k, b.ring_v, b.ring_len, b.k_fwd[j], b.v_fwd[j],
+                                         b.n_sink, b.window, b.sm_scale, b.ws, out=b.out["fwd"],
+                                         lse=b.out["fwd_lse"])
 
     def draft_native(self, log: Optional[CallLog] = None):
         b, s = self.b, self.s

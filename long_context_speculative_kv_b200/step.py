@@ -6,6 +6,8 @@ identity (Pith verdict on arXiv 2607.21535, pith_extraction.key_machinery, Eq. 1
   * t_ctx_draft: append the gamma + 1 committed tokens' draft K/V, then one draft attention call
     with n_q = gamma + 1 (worst case: every draft of the previous step accepted);
   * t_fwd_draft: append one draft K/V row, then one draft attention call with n_q = 1;
+    in the windowed arm each of these pairs is one library call (draft_attn_window_append: the
+    append happens inside the attention kernel);
   * t_verify:    one verify_attn call per target attention layer (n_q = gamma + 1, or the tree);
   * acceptance:  accept_greedy over the verify step's logits.
 
@@ -106,20 +108,27 @@ class DecodeStep:
             Hkv = bufs.k_pools[0].shape[1]
             need = max(api.workspace_bytes(B, max(n_q, gamma + 1), Hq, Hkv),
                        api.workspace_bytes(B, 1, Hq, Hkv))
-            b.ws = torch.empty(need, dtype=torch.uint8, device=bufs.q_verify.device)
+            b.ws = torch.zeros(need, dtype=torch.uint8, device=bufs.q_verify.device)
 
     # ----------------------------------------------------------------------------- phases
     def draft_windowed(self, log: Optional[CallLog] = None):
         b = self.b
-        if log: log.mark("append_ctx")
-        self._append(b.k_ctx, b.v_ctx)
         if log: log.mark("window_ctx")
-        self._window(b.q_ctx, b.out["ctx"], b.out["ctx_lse"])
+        self._forward(b.q_ctx, b.k_ctx, b.v_ctx, b.out["ctx"], b.out["ctx_lse"])
         for j in range(self.gamma):
-            if log: log.mark("append_fwd")
-            self._append(b.k_fwd[j], b.v_fwd[j])
             if log: log.mark("window_fwd")
-            self._window(b.q_fwd[j], b.out["fwd"], b.out["fwd_lse"])
+            self._forward(b.q_fwd[j], b.k_fwd[j], b.v_fwd[j], b.out["fwd"], b.out["fwd_lse"])
+
+    def _forward(self, q, k_new, v_new, out, lse):
+        """Ring append of the new rows and the windowed attention, one library call."""
+        b = self.b
+        if b.kv8:
+            api.draft_attn_window_append_fp8(q, b.ring_k, b.ring_v, b.ring_len, k_new, v_new, b.n_sink,
+                                             b.window, b.sm_scale, b.k_scale, b.v_scale, b.ws,
+                                             out=out, lse=lse)
+        else:
+            api.draft_attn_window_append(q, b.ring_k, b.ring_v, b.ring_len, k_new, v_new, b.n_sink,
+                                         b.window, b.sm_scale, b.ws, out=out, lse=lse)
 
     def _append(self, k_new, v_new):
         b = self.b

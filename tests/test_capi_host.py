@@ -35,7 +35,8 @@ def test_header_declares_the_five_calls_and_helpers():
             "wmtp_device_status", "wmtp_launch_count", "draft_attn_window_noalloc",
             "accept_stochastic", "ring_kv_append_at", "spec_commit", "ring_kv_append_fp8",
             "draft_attn_window_fp8", "draft_attn_full_fp8", "verify_attn_fp8", "wmtp_synth_draft_tokens",
-            "wmtp_synth_target_logits", "wmtp_selftest_wait_timeout"} == names
+            "wmtp_synth_target_logits", "wmtp_selftest_wait_timeout", "draft_attn_window_append",
+            "draft_attn_window_append_fp8"} == names
     assert set(_lib._SIGNATURES) == names
 
 
@@ -96,6 +97,27 @@ def test_attention_host_checks(lib):
     v = lib.verify_attn
     assert v(GOOD, GOOD, GOOD, GOOD, GOOD, BAD, 1, 4, 8, 2, 128, 64, 4, 4, 1.0, GOOD, None, GOOD, 1 << 30, None) == -3
     assert v(GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, 4, 8, 2, 128, 64, 4, 4, 1.0, GOOD, None, GOOD, 1 << 30, None) == -1
+
+
+def test_window_append_host_checks(lib):
+    f = lib.draft_attn_window_append
+    # (q, rk, rv, rlen, k_new, v_new, n_new, B, n_q, Hq, Hkv, D, s, W, C, scale, out, lse, ws, n, stream)
+    ok = (GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 1, 1, 1, 8, 2, 128, 4, 252, 256, 1.0, GOOD, None, GOOD, 1 << 30, None)
+
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[int(k[1:])] = v
+        return f(*a)
+    assert call(a6=-1) == -1                          # n_new < 0
+    assert call(a4=None) == -1                        # k_new missing with n_new > 0
+    assert call(a5=BAD) == -3                         # v_new misaligned
+    assert call(a3=ctypes.c_void_p(0x10004)) == -3    # ring_len not 8-byte aligned
+    assert call(a10=3) == -2                          # Hq % Hkv != 0
+    assert call(a13=253) == -1                        # window > capacity - n_sink
+    g = lib.draft_attn_window_append_fp8
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 1, 1, 1, 8, 2, 128, 4, 252, 256, 1.0, -1.0, 1.0,
+             GOOD, None, GOOD, 1 << 30, None) == -1   # k_scale <= 0
 
 
 def test_selftest_wait_limit_checked_on_host(lib):

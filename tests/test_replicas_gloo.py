@@ -1,6 +1,7 @@
 """The multi-GPU path is replicas only (no exchange step): world-size-2 checks of the benchmark's
 cross-rank logic on CPU with the gloo backend -- the max-over-ranks timing reduction every rank
-takes part in, the whole-job aggregate, and the reference arm's rank-0-only rule."""
+takes part in, the per-replica step time and the whole-job throughput taken from it, and the
+reference arm's rank-0-only rule."""
 import os
 import socket
 
@@ -23,7 +24,7 @@ def _worker(rank: int, world: int, port: int, out):
     try:
         ms = [12.5, 17.25][rank]                     # each replica's own timed-region length
         m = bench.max_over_ranks(ms, world)
-        out[rank] = (m, bench.aggregate_us_per_step(m, 10, world))
+        out[rank] = (m, bench.per_replica_us_per_step(m, 10), bench.aggregate_steps_per_s(m, 10, world))
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -37,14 +38,16 @@ def test_max_over_ranks_and_aggregate_with_two_gloo_ranks():
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
     for rank in range(world):
-        m, agg = res[rank]
+        m, per_step, agg = res[rank]
         assert m == 17.25                            # the slowest rank's time, on every rank
-        assert agg == pytest.approx(17.25e3 / (10 * 2))
+        assert per_step == pytest.approx(17.25e3 / 10)    # a replica's step latency
+        assert agg == pytest.approx(10 * 2 / 17.25e-3)    # decode steps per second, whole job
 
 
 def test_single_rank_reduction_is_identity():
     assert bench.max_over_ranks(3.5, 1) == 3.5
-    assert bench.aggregate_us_per_step(2.0, 4, 1) == 500.0
+    assert bench.per_replica_us_per_step(2.0, 4) == 500.0
+    assert bench.aggregate_steps_per_s(2.0, 4, 1) == pytest.approx(2000.0)
 
 
 def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
