@@ -468,90 +468,105 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         }
     } else if (KV8 && warp >= 12) {
         // =========================== converters (fp8 KV) =====================================
-        // Pair 0 (warps 12-13) takes the even tiles, pair 1 (warps 14-15) the odd ones.  Thread r
-        // of a pair owns key row r of its V tiles (widened to fp16 in place) and, at a unit's
-        // first tile, query row r of the unit (split in place into the E4M3 hi and lo terms).
+        // Pair 0 (warps 12-13) takes the even tiles, pair 1 (warps 14-15) the odd ones; NV is
+        // even, so each V slot belongs to one pair and its phases are waited on in order.  Thread
+        // r of a pair owns key row r of its V tiles (widened to fp16 in place).  Pair 0 also
+        // splits every unit's bf16 Q rows into the E4M3 hi / lo terms, strictly in unit order
+        // (before its tile t it converts every unit up to tile t's), so its waits on the Q
+        // buffers' phases are in order too: unit u + 2's Q cannot land before unit u is
+        // converted (its buffer is freed only after unit u's last QK^T).
+        static_assert(!KV8 || NV % 2 == 0, "each V slot belongs to one converter pair");
         const uint32_t pair = (uint32_t)(warp - 12) >> 1;
         const int r = threadIdx.x - 384 - 64 * (int)pair;            // 0 .. 63
+        // Splits unit u's Q row r in place (the unit's rows form one row block of <= 64 rows).
+        auto convert_q = [&](uint32_t u) -> bool {
+            const uint32_t qb = u & 1u;
+            if (!mbar_wait_bounded(&q_full[qb], (u >> 1) & 1u)) return false;
+            const uint32_t row = smem_addr(smem + L::kQOff + qb * L::kQBytes) + (uint32_t)(r * 128);
+            const bool live = r < a.rows_total;
+            // chunk c of the bf16 boxes (box c / 8): dims 8 c .. 8 c + 7 of the row
+            auto bchunk = [&](int c) -> uint32_t {
+                return row + (uint32_t)((c >> 3) * kHalfBytes) + (uint32_t)(((c & 7) ^ (r & 7)) << 4);
+            };
+            float amax = 0.f;
+            if (live) {
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t w4[4];
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3]) : "r"(bchunk(c)) : "memory");
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[k] << 16)),
+                                                 fabsf(__uint_as_float(w4[k] & 0xffff0000u))));
+                }
+            }
+            // 2^k q < 2^8 for the row's largest |q| (E4M3 reaches 448); the row's scores come out
+            // 2^k too large, so its softmax scale carries 2^-k
+            int e = 0;
+            if (amax > 0.f) (void)frexpf(amax, &e);
+            const int k2 = 8 - e;
+            const float up = ldexpf(1.f, k2);
+            qscale[(u % L::kQScaleRing) * 64 + r] = ldexpf(a.scale_log2, -k2);
+            // output chunk c holds the codes of dims 16 c .. 16 c + 15 (lowest dim in the lowest
+            // byte): hi in chunk c of box 0's space, lo in chunk c of box 1's space.  Writing hi
+            // chunk c clobbers bf16 dims 8 c .. of box 0, which output chunks <= c have read
+            // already; the lo chunks would clobber box 1 dims still unread, so they are held in
+            // registers and written last.
+            uint32_t lo[8][4];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w8[8];
+                if (live) {
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w8[0]), "=r"(w8[1]), "=r"(w8[2]), "=r"(w8[3]) : "r"(bchunk(2 * c)) : "memory");
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w8[4]), "=r"(w8[5]), "=r"(w8[6]), "=r"(w8[7]) : "r"(bchunk(2 * c + 1)) : "memory");
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) w8[k] = 0u;
+                }
+                uint32_t hi4[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t wa = w8[2 * k], wb = w8[2 * k + 1];
+                    const float x0 = __uint_as_float(wa << 16) * up;
+                    const float x1 = __uint_as_float(wa & 0xffff0000u) * up;
+                    const float x2 = __uint_as_float(wb << 16) * up;
+                    const float x3 = __uint_as_float(wb & 0xffff0000u) * up;
+                    hi4[k] = f32x2_to_e4m3x2(x0, x1) | (f32x2_to_e4m3x2(x2, x3) << 16);
+                    uint32_t h01, h23;
+                    e4m3x4_to_f16x2x2(hi4[k], h01, h23);
+                    const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                    const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                    lo[c][k] = f32x2_to_e4m3x2(x0 - v01.x, x1 - v01.y) |
+                               (f32x2_to_e4m3x2(x2 - v23.x, x3 - v23.y) << 16);
+                }
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                             :: "r"(row + (uint32_t)((c ^ (r & 7)) << 4)), "r"(hi4[0]), "r"(hi4[1]),
+                                "r"(hi4[2]), "r"(hi4[3]) : "memory");
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                             :: "r"(row + (uint32_t)kHalfBytes + (uint32_t)((c ^ (r & 7)) << 4)),
+                                "r"(lo[c][0]), "r"(lo[c][1]), "r"(lo[c][2]), "r"(lo[c][3]) : "memory");
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_conv[qb]);
+            return true;
+        };
+        uint32_t next_u = 0;                                         // pair 0: next unit to split
+        bool qok = true;
+        TileMeta last{};
         for (uint32_t t = pair; t < n; t += 2) {
             const uint32_t vs = t % NV;
             if (!mbar_wait_bounded(&v8full[vs], (t / NV) & 1u)) break;
             const TileMeta m = vmeta[vs];
-            if (m.flags & kFirst) {
-                const uint32_t u = (uint32_t)m.ord, qb = u & 1u;
-                if (!mbar_wait_bounded(&q_full[qb], (u >> 1) & 1u)) break;
-                const uint32_t row = smem_addr(smem + L::kQOff + qb * L::kQBytes) + (uint32_t)(r * 128);
-                const bool live = r < a.rows_total - m.rb * kRowsPerBlock;
-                // chunk c of the bf16 boxes (box c / 8): dims 8 c .. 8 c + 7 of the row
-                auto bchunk = [&](int c) -> uint32_t {
-                    return row + (uint32_t)((c >> 3) * kHalfBytes) + (uint32_t)(((c & 7) ^ (r & 7)) << 4);
-                };
-                float amax = 0.f;
-                if (live) {
-#pragma unroll 4
-                    for (int c = 0; c < 16; ++c) {
-                        uint32_t w4[4];
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3]) : "r"(bchunk(c)) : "memory");
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[k] << 16)),
-                                                     fabsf(__uint_as_float(w4[k] & 0xffff0000u))));
-                    }
-                }
-                // 2^k q < 2^8 for the row's largest |q| (E4M3 reaches 448); the row's scores come
-                // out 2^k too large, so its softmax scale carries 2^-k
-                int e = 0;
-                if (amax > 0.f) (void)frexpf(amax, &e);
-                const int k2 = 8 - e;
-                const float up = ldexpf(1.f, k2);
-                qscale[(u % L::kQScaleRing) * 64 + r] = ldexpf(a.scale_log2, -k2);
-                // output chunk c holds the codes of dims 16 c .. 16 c + 15 (lowest dim in the lowest
-                // byte): hi in chunk c of box 0's space, lo in chunk c of box 1's space.  Writing hi
-                // chunk c clobbers bf16 dims 8 c .. of box 0, which output chunks <= c have read
-                // already; the lo chunks would clobber box 1 dims still unread, so they are held
-                // in registers and written last.
-                uint32_t lo[8][4];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t w8[8];
-                    if (live) {
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(w8[0]), "=r"(w8[1]), "=r"(w8[2]), "=r"(w8[3]) : "r"(bchunk(2 * c)) : "memory");
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(w8[4]), "=r"(w8[5]), "=r"(w8[6]), "=r"(w8[7]) : "r"(bchunk(2 * c + 1)) : "memory");
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) w8[k] = 0u;
-                    }
-                    uint32_t hi4[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t wa = w8[2 * k], wb = w8[2 * k + 1];
-                        const float x0 = __uint_as_float(wa << 16) * up;
-                        const float x1 = __uint_as_float(wa & 0xffff0000u) * up;
-                        const float x2 = __uint_as_float(wb << 16) * up;
-                        const float x3 = __uint_as_float(wb & 0xffff0000u) * up;
-                        hi4[k] = f32x2_to_e4m3x2(x0, x1) | (f32x2_to_e4m3x2(x2, x3) << 16);
-                        uint32_t h01, h23;
-                        e4m3x4_to_f16x2x2(hi4[k], h01, h23);
-                        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-                        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-                        lo[c][k] = f32x2_to_e4m3x2(x0 - v01.x, x1 - v01.y) |
-                                   (f32x2_to_e4m3x2(x2 - v23.x, x3 - v23.y) << 16);
-                    }
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                                 :: "r"(row + (uint32_t)((c ^ (r & 7)) << 4)), "r"(hi4[0]), "r"(hi4[1]),
-                                    "r"(hi4[2]), "r"(hi4[3]) : "memory");
-                }
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                                 :: "r"(row + (uint32_t)kHalfBytes + (uint32_t)((c ^ (r & 7)) << 4)),
-                                    "r"(lo[c][0]), "r"(lo[c][1]), "r"(lo[c][2]), "r"(lo[c][3]) : "memory");
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&q_conv[qb]);
+            last = m;
+            if (pair == 0u) {
+                while (qok && next_u <= (uint32_t)m.ord) qok = convert_q(next_u++);
+                if (!qok) break;
             }
             // rows past the valid keys come out as zeros (codes there may be anything)
             const uint32_t base = smem_addr(smem + L::kVOff + vs * kTileBytes);
@@ -560,6 +575,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&vfull[vs]);
         }
+        // pair 0's last tile (n - 2) ended its unit: tile n - 1 starts one more unit
+        if (pair == 0u && qok && n >= 2 && (n & 1u) == 0u && (last.flags & kLast) &&
+            next_u == (uint32_t)last.ord + 1u)
+            (void)convert_q(next_u);
     } else {
         // =========================== softmax warps (two groups) ==============================
         const uint32_t grp = warp >= 8 ? 1u : 0u;

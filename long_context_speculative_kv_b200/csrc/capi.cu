@@ -226,7 +226,7 @@ int set_smem_once(K kern, int bytes, bool (&done)[kMaxDevices]) {
 //         > 64 rows       mma.sync (4, 1, 2 stages, 2 CTAs/SM) per 64-row block
 //   fp8   rows <= 16      mma.sync, Q in shared memory (1, 4, 2 stages, 3 CTAs/SM)   0.82
 //         rows 17..32     mma.sync (2, 2, 4 stages, 2 CTAs/SM)
-//         rows 33..64     tcgen05 with converter warps
+//         rows 33..64     tcgen05: QK^T on the E4M3 key codes, V widened by converter warps
 //         > 64 rows       mma.sync (4, 1, 4 stages, 2 CTAs/SM) per 64-row block
 // The 1-CTA mma.sync layouts above 16 rows were latency-bound (one consumer warp per SM
 // sub-partition); two independent CTA pipelines per SM fixed that.  The tcgen05 kernel needs
@@ -302,7 +302,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
         case Kern::kSplit16Fp8: return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);
         case Kern::kSplit32Fp8: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
         case Kern::kSplit64Fp8: return launch_attn_t<SRC, 4, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
-        case Kern::kTcFp8: return launch_attn_tc_t<SRC, 3, 3, 2, true>(km, vm, a.q, a, sm_count, s, st);
+        case Kern::kTcFp8: return launch_attn_tc_t<SRC, 4, 4, 2, true>(km, vm, a.q, a, sm_count, s, st);
     }
     return WMTP_ERR_ARG;
 }
