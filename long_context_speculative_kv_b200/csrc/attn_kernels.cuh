@@ -349,6 +349,7 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* s
     using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
     constexpr int kWarps = NMT * NKG + 1;
     cluster_sync_all();
+    if (warp == 0 && lane == 0) WMTP_TRACE_AT(29);
     const int cs = (int)gridDim.x, me = (int)blockIdx.x;
     const int rows_u = min(kRowsPerBlock, a.rows_total - wk.rb * kRowsPerBlock);
     const uint32_t part = smem_addr(smem + L::kPartOff);
@@ -382,6 +383,7 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* s
         *reinterpret_cast<uint2*>(a.out + orow * kD + 4 * lane) = pk;
         if (a.lse != nullptr && lane == 0) a.lse[orow] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
     }
+    if (warp == 0 && lane == 0) WMTP_TRACE_AT(30);
     __syncwarp();
     cluster_sync_all();
 }
@@ -438,12 +440,14 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    if (threadIdx.x == 0) WMTP_TRACE_AT(0);
     pdl_launch_dependents();
     if (warp == NWC && lane == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
     pdl_wait();
+    if (threadIdx.x == 0) WMTP_TRACE_AT(1);
 
     __shared__ RingUnitWalker s_walk;          // cluster mode: this CTA's unit
     // ---- plan: lengths -> tiles per request -> this CTA's tile range ------------------------
@@ -510,6 +514,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         }
     }
     __syncthreads();
+    if (threadIdx.x == 0) WMTP_TRACE_AT(2);
     const long long t_begin = s_range[0], t_end = s_range[1];
     if (!CL && t_begin >= t_end) return;
 
@@ -545,6 +550,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 } else {
                     mbar_arrive(&full_bar[stage]);
                 }
+                if (it < 8) WMTP_TRACE_AT(3 + (int)it);
             }
             // Drain: wait (bounded) until the consumers released every stage, so no TMA copy is
             // in flight into this CTA's shared memory when it exits.
@@ -600,6 +606,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         const int stage = (int)(it % NSTAGE);
         const uint32_t phase = (it / NSTAGE) & 1u;
         if (!mbar_wait_bounded(&full_bar[stage], phase)) { alive = false; break; }
+        if (warp == 0 && lane == 0 && it < 8) WMTP_TRACE_AT(12 + (int)it);
         const TileMeta m = meta[stage];
         bool patched = false;
         if (CL && a.n_new > 0 && m.nvalid > 0) {
@@ -715,6 +722,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             }
         }
 
+        if (warp == 0 && lane == 0 && (m.flags & kFirst)) WMTP_TRACE_AT(11);
         if (m.nvalid > 0) {
             const uint32_t kbase = smem_addr(smem + (size_t)stage * kStage);
             const uint32_t vbase = kbase + (KV8 ? kTileBytes8 : kTileBytes);
@@ -823,10 +831,11 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     const float p1 = fast_exp2(fmaf(s[n][2 * r + 1], a.scale_log2, -m_use[r]));
                     uint32_t pk;
                     if (KV8) {
-                        // fp16 weights; the row sum uses the same rounded weights
+                        // fp16 weights; the row sum over the fp32 weights (fp16 keeps 11 bits: the
+                        // two sums differ far below the tolerance, and the conversions back would
+                        // compete with the key / value widening for the conversion pipe)
                         pk = pack_f16x2(p0, p1);
-                        const float2 pr = __half22float2(*reinterpret_cast<const __half2*>(&pk));
-                        l_r[r] += pr.x + pr.y;
+                        l_r[r] += p0 + p1;
                     } else {
                         pk = pack_bf16x2(p0, p1);
                         // the row sum uses the same bf16-rounded weights the PV product uses
@@ -895,6 +904,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         if (CL && patched) fence_proxy_async();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
+        if (warp == 0 && lane == 0 && it < 8) WMTP_TRACE_AT(20 + (int)it);
 
         if (m.flags & kLast) {
             // ---- unit end: combine key groups, then write the result or a partial ----------
@@ -1032,9 +1042,11 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             }
         }
     }
+    if (warp == 0 && lane == 0) WMTP_TRACE_AT(28);
     if (CL) {
         __syncwarp();
         cluster_merge_rows<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
+        if (warp == 0 && lane == 0) WMTP_TRACE_AT(31);
     }
 }
 

@@ -682,10 +682,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 const float p0 = fast_exp2(fmaf(x[2 * j], rs, -m_sub));
                 const float p1 = fast_exp2(fmaf(x[2 * j + 1], rs, -m_sub));
                 if (KV8) {
-                    // fp16 weights for the fp16 V; the row sum over the same rounded weights
+                    // fp16 weights for the fp16 V; the row sum over the fp32 weights (fp16 keeps 11
+                    // bits, so the two sums differ by far less than the tolerance, and the
+                    // conversions back to fp32 would compete with the V widening for the
+                    // conversion pipe)
                     pk[j] = pack_f16x2(p0, p1);
-                    const float2 pr = __half22float2(*reinterpret_cast<const __half2*>(&pk[j]));
-                    ls[j & 3] += pr.x + pr.y;
+                    ls[j & 3] += p0 + p1;
                 } else {
                     pk[j] = pack_bf16x2(p0, p1);
                     ls[j & 3] += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);

@@ -225,19 +225,19 @@ int set_smem_once(K kern, int bytes, bool (&done)[kMaxDevices]) {
 //         rows 33..64     tcgen05 / TMEM (K pair slots 3, V ring 3, S buffers 2)     0.96
 //         > 64 rows       mma.sync (4, 1, 2 stages, 2 CTAs/SM) per 64-row block
 //   fp8   rows <= 16      mma.sync, Q in shared memory (1, 4, 2 stages, 3 CTAs/SM)   0.82
-//         rows 17..32     mma.sync (2, 2, 4 stages, 2 CTAs/SM)
-//         rows 33..64     tcgen05: QK^T on the E4M3 key codes, V widened by converter warps
+//         rows 17..64     tcgen05: QK^T on the E4M3 key codes, V widened by converter warps
 //         > 64 rows       mma.sync (4, 1, 4 stages, 2 CTAs/SM) per 64-row block
 // The 1-CTA mma.sync layouts above 16 rows were latency-bound (one consumer warp per SM
 // sub-partition); two independent CTA pipelines per SM fixed that.  The tcgen05 kernel needs
 // the whole unit in one 64-row block (its Q arrives as one TMA box of n_q x G rows).
-// Build-time option for measurement sweeps: the smallest unit (in rows) the tcgen05 kernel takes,
-// bf16 and fp8 KV (default 33 for both).
+// Build-time option for measurement sweeps: the smallest unit (in rows) the tcgen05 kernel takes
+// (bf16: 33, where the mma.sync layouts fall behind; fp8: 17, the tcgen05 kernel's QK^T on the
+// key codes beats the register-widening layout from 17 rows, 318 vs 338 us at 1M keys, 32 rows).
 #ifndef WMTP_TC_MIN_ROWS
 #define WMTP_TC_MIN_ROWS 33
 #endif
 #ifndef WMTP_TC8_MIN_ROWS
-#define WMTP_TC8_MIN_ROWS 33
+#define WMTP_TC8_MIN_ROWS 17
 #endif
 enum class Kern { kSplit16, kSplit32, kSplit64, kTc, kSplit16Fp8, kSplit32Fp8, kSplit64Fp8, kTcFp8 };
 
@@ -343,6 +343,18 @@ int cluster_capacity(K kern, int smem, int threads, int cs, int (&cache)[kMaxDev
     return cache[dev][k];
 }
 
+// Build-time options for measurement sweeps: the largest cluster size, and the stage count /
+// CTAs per SM of the layout for units of at most 16 rows.
+#ifndef WMTP_CL_MAX
+#define WMTP_CL_MAX 16
+#endif
+#ifndef WMTP_CL16_NSTAGE
+#define WMTP_CL16_NSTAGE 4
+#endif
+#ifndef WMTP_CL16_MINB
+#define WMTP_CL16_MINB 1
+#endif
+
 template <int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
 int launch_window_cluster_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
                             const Shape& s, int max_tiles, cudaStream_t st) {
@@ -364,27 +376,30 @@ int launch_window_cluster_t(const CUtensorMap& km, const CUtensorMap& vm, const 
         }
     }
     int cs = 1;
-    for (int c = 16; c >= 2; c >>= 1) {
+    for (int c = WMTP_CL_MAX; c >= 2; c >>= 1) {
         if (2 * c > max_tiles) continue;
         const int n = cluster_capacity(kern, Lay::kAlloc, kThreads, c, cap, cap_init);
         if (n > 0 && s.units <= n) { cs = c; break; }
     }
+#ifdef WMTP_CL_REPORT
+    std::fprintf(stderr, "[wmtp] window cluster: units %d, size %d, %d threads, %d bytes shared\n",
+                 s.units, cs, kThreads, Lay::kAlloc);
+#endif
     return launch_cluster(kern, dim3(cs, s.units), dim3(kThreads), Lay::kAlloc, st, cs, km, vm, a);
 }
 
 int launch_window_cluster(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
                           const Shape& s, int max_tiles, cudaStream_t st, bool kv8) {
-    switch (select_kernel(s, kv8)) {
-        case Kern::kSplit16: return launch_window_cluster_t<1, 4, 4, 1>(km, vm, a, s, max_tiles, st);
-        case Kern::kSplit32: return launch_window_cluster_t<2, 2, 2, 2>(km, vm, a, s, max_tiles, st);
-        case Kern::kSplit64: case Kern::kTc:
-            return launch_window_cluster_t<4, 1, 2, 2>(km, vm, a, s, max_tiles, st);
-        case Kern::kSplit16Fp8: return launch_window_cluster_t<1, 4, 2, 3, true, true>(km, vm, a, s, max_tiles, st);
-        case Kern::kSplit32Fp8: return launch_window_cluster_t<2, 2, 4, 2, true>(km, vm, a, s, max_tiles, st);
-        case Kern::kSplit64Fp8: case Kern::kTcFp8:
-            return launch_window_cluster_t<4, 1, 4, 2, true>(km, vm, a, s, max_tiles, st);
-    }
-    return WMTP_ERR_ARG;
+    // the mma.sync layouts of the stream-K kernel, by the unit's rows (the windowed units are
+    // short, so the tcgen05 kernel's deeper pipeline does not pay here)
+    if (s.rows_blk <= 16)
+        return kv8 ? launch_window_cluster_t<1, 4, 2, 3, true, true>(km, vm, a, s, max_tiles, st)
+                   : launch_window_cluster_t<1, 4, WMTP_CL16_NSTAGE, WMTP_CL16_MINB>(km, vm, a, s, max_tiles, st);
+    if (s.rows_blk <= 32)
+        return kv8 ? launch_window_cluster_t<2, 2, 4, 2, true>(km, vm, a, s, max_tiles, st)
+                   : launch_window_cluster_t<2, 2, 2, 2>(km, vm, a, s, max_tiles, st);
+    return kv8 ? launch_window_cluster_t<4, 1, 4, 2, true>(km, vm, a, s, max_tiles, st)
+               : launch_window_cluster_t<4, 1, 2, 2>(km, vm, a, s, max_tiles, st);
 }
 
 // Common front half of the three attention calls.
@@ -869,6 +884,16 @@ int wmtp_synth_target_logits(const int32_t* history, const int64_t* n_tokens, in
 }
 
 uint64_t wmtp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+#ifdef WMTP_TRACE
+// Measurement builds only: copies the timestamp trace of CTA (0, 0) of the last traced launch.
+WMTP_API int wmtp_trace_read(unsigned long long* host, int n) {
+    if (host == nullptr || n < 1 || n > kTraceSlots) return WMTP_ERR_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return WMTP_ERR_CUDA;
+    return cudaMemcpyFromSymbol(host, g_trace, sizeof(unsigned long long) * n) == cudaSuccess ? WMTP_OK
+                                                                                            : WMTP_ERR_CUDA;
+}
+#endif
 
 int wmtp_selftest_wait_timeout(uint64_t limit_ns, wmtp_stream_t stream) {
     if (limit_ns < 1000000ull || limit_ns > kWaitLimitNs) return WMTP_ERR_ARG;

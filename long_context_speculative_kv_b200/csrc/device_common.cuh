@@ -35,6 +35,21 @@ __device__ __forceinline__ uint64_t global_ns() {
 // kernel return.  Healthy waits last microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
+// Build-time timestamp trace for measurement (off unless WMTP_TRACE is defined): named points of
+// CTA (0, 0) record the global timer; read with wmtp_trace_read.
+#ifdef WMTP_TRACE
+constexpr int kTraceSlots = 64;
+__device__ unsigned long long g_trace[kTraceSlots];
+#define WMTP_TRACE_AT(i)                                                            \
+    do {                                                                            \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && (i) < kTraceSlots) g_trace[(i)] = global_ns(); \
+    } while (0)
+#else
+#define WMTP_TRACE_AT(i) \
+    do {                 \
+    } while (0)
+#endif
+
 // ---------------------------------------------------------------------------------------------
 // mbarrier (shared::cta).
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

@@ -120,8 +120,9 @@ def test_more_new_rows_than_the_window():
     rl = [torch.zeros(B, dtype=torch.int64, device="cuda") for _ in range(2)]
     for i in range(2):
         api.ring_kv_append(rings[i][0], rings[i][1], rl[i], to_dev_bf16(k_tok[:, :L0]), to_dev_bf16(v_tok[:, :L0]), s)
-    q_bits = gen.normal_bf16(rng, (B, n_new, Hq, D))
-    ws = api.alloc_workspace(B, n_new, Hq, Hkv)
+    n_q = 2                                            # queries at the last two positions
+    q_bits = gen.normal_bf16(rng, (B, n_q, Hq, D))
+    ws = api.alloc_workspace(B, n_q, Hq, Hkv)
     kn, vn = to_dev_bf16(k_tok[:, L0:]), to_dev_bf16(v_tok[:, L0:])
     out, lse = api.draft_attn_window_append(to_dev_bf16(q_bits), rings[0][0], rings[0][1], rl[0], kn, vn, s, W,
                                             sc, ws)
