@@ -365,12 +365,20 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* s
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float wsum = 0.f;
         const uint32_t po = part + 4u * (uint32_t)(rr * kD + 4 * lane);
-        for (int k = 0; k < cs; ++k) {
-            const float wk_ = __shfl_sync(0xffffffffu, w, k);
-            if (wk_ > 0.f) {
-                const float4 v = ld_dsmem_v4(map_shared_rank(po, k));
-                acc.x += wk_ * v.x; acc.y += wk_ * v.y; acc.z += wk_ * v.z; acc.w += wk_ * v.w;
-                wsum += wk_;
+        // eight ranks' loads in flight at a time (a load waited on before the next is issued
+        // would cost one distributed-shared-memory round trip per rank)
+        for (int k0 = 0; k0 < cs; k0 += 8) {
+            float4 v[8];
+            float wv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                wv[j] = (k0 + j < cs) ? __shfl_sync(0xffffffffu, w, k0 + j) : 0.f;
+                v[j] = wv[j] > 0.f ? ld_dsmem_v4(map_shared_rank(po, (uint32_t)(k0 + j))) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                acc.x += wv[j] * v[j].x; acc.y += wv[j] * v[j].y; acc.z += wv[j] * v[j].z; acc.w += wv[j] * v[j].w;
+                wsum += wv[j];
             }
         }
         const int R = wk.rb * kRowsPerBlock + rr;
@@ -543,14 +551,20 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     tma_load_3d(st + kTileBytes8, &vmap, &full_bar[stage], 0, ty, tz, pol);
                 } else if (m.nvalid > 0) {
                     mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+#ifdef WMTP_TMA4D
+                    // one box per tensor: (64 dims, 64 rows, 2 halves) lands as [half][row][64]
+                    tma_load_4d_hint(st, &kmap, &full_bar[stage], 0, ty, 0, tz, pol);
+                    tma_load_4d_hint(st + kTileBytes, &vmap, &full_bar[stage], 0, ty, 0, tz, pol);
+#else
                     tma_load_3d(st, &kmap, &full_bar[stage], 0, ty, tz, pol);
                     tma_load_3d(st + kHalfBytes, &kmap, &full_bar[stage], 64, ty, tz, pol);
                     tma_load_3d(st + kTileBytes, &vmap, &full_bar[stage], 0, ty, tz, pol);
                     tma_load_3d(st + kTileBytes + kHalfBytes, &vmap, &full_bar[stage], 64, ty, tz, pol);
+#endif
                 } else {
                     mbar_arrive(&full_bar[stage]);
                 }
-                if (it < 8) WMTP_TRACE_AT(3 + (int)it);
+                WMTP_TRACE_TILE(0, it);
             }
             // Drain: wait (bounded) until the consumers released every stage, so no TMA copy is
             // in flight into this CTA's shared memory when it exits.
@@ -602,11 +616,99 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         sync_phase ^= 1u;
         return ok;
     };
+    // Unit start: this warp's Q rows, the rows' visibility masks, state reset.  Returns false
+    // when a bounded rendezvous gave up.
+    auto unit_start = [&](const TileMeta& m) -> bool {
+            // ---- unit start: load this warp's Q rows, visibility masks, reset state -------
+            Lpre = m.L_tot - a.n_q;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
+                row_ok[r] = R < a.rows_total;
+                const int i = row_ok[r] ? R / a.G : 0;
+                vis[r] = step_visibility(a, m.b, i);
+                m_r[r] = -INFINITY;
+                l_r[r] = 0.f;
+            }
+#pragma unroll
+            for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            if constexpr (QS) {
+                // every warp is past the previous unit's reads of these rows; each consumer thread
+                // widens quarter rows (32 dims) of the unit's Q into shared memory
+                if (!consumers_sync()) return false;
+                for (int w = threadIdx.x; w < NMT * 16 * 4; w += NWC * 32) {
+                    const int row = w >> 2, part = w & 3;
+                    const int R = m.rb * kRowsPerBlock + row;
+                    uint32_t h[16];
+                    if (R < a.rows_total) {
+                        const int i = R / a.G, g = R - (R / a.G) * a.G;
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD + 32 * part);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint4 v = __ldg(src + k);
+                            h[4 * k] = bf16x2_to_f16x2(v.x);
+                            h[4 * k + 1] = bf16x2_to_f16x2(v.y);
+                            h[4 * k + 2] = bf16x2_to_f16x2(v.z);
+                            h[4 * k + 3] = bf16x2_to_f16x2(v.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) h[k] = 0u;
+                    }
+                    const uint32_t dst = smem_addr(smem + L::kQOff) + (uint32_t)(row * L::kQStride + 64 * part);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                                     :: "r"(dst + 16u * k), "r"(h[4 * k]), "r"(h[4 * k + 1]),
+                                        "r"(h[4 * k + 2]), "r"(h[4 * k + 3]) : "memory");
+                }
+                if (!consumers_sync()) return false;
+            } else {
+            const uint32_t* q32[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
+                const int i = R / a.G, g = R - (R / a.G) * a.G;
+                q32[r] = reinterpret_cast<const uint32_t*>(
+                    a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD);
+            }
+            if (KV8) {
+                // fp16 A-fragments with the k order of the fp8 K fragments: k slots (2 tig, +1)
+                // and (2 tig + 8, +9) of step ks hold dims 16 ks + 4 tig + (0, 1) and (2, 3)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int c = ks * 8 + 2 * tig;
+                    qa[ks][0] = row_ok[0] ? bf16x2_to_f16x2(__ldg(q32[0] + c)) : 0u;
+                    qa[ks][1] = row_ok[1] ? bf16x2_to_f16x2(__ldg(q32[1] + c)) : 0u;
+                    qa[ks][2] = row_ok[0] ? bf16x2_to_f16x2(__ldg(q32[0] + c + 1)) : 0u;
+                    qa[ks][3] = row_ok[1] ? bf16x2_to_f16x2(__ldg(q32[1] + c + 1)) : 0u;
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int c = ks * 8 + tig;     // 32-bit word index of dims (16 ks + 2 tig)
+                    qa[ks][0] = row_ok[0] ? __ldg(q32[0] + c) : 0u;
+                    qa[ks][1] = row_ok[1] ? __ldg(q32[1] + c) : 0u;
+                    qa[ks][2] = row_ok[0] ? __ldg(q32[0] + c + 4) : 0u;
+                    qa[ks][3] = row_ok[1] ? __ldg(q32[1] + c + 4) : 0u;
+                }
+            }
+            }
+                return true;
+    };
+    if (CL && t_begin < t_end) {
+        // cluster mode: the unit is known from the plan, so its Q loads overlap the first tile's
+        TileMeta m0;
+        int ty0 = 0, tz0 = 0;
+        s_walk.describe(a, (int)t_begin, (int)t_begin, (int)t_end, m0, ty0, tz0);
+        if (!unit_start(m0)) alive = false;
+    }
     for (long long t = t_begin; t < t_end && alive; ++t, ++it) {
         const int stage = (int)(it % NSTAGE);
         const uint32_t phase = (it / NSTAGE) & 1u;
         if (!mbar_wait_bounded(&full_bar[stage], phase)) { alive = false; break; }
-        if (warp == 0 && lane == 0 && it < 8) WMTP_TRACE_AT(12 + (int)it);
+        if (warp == 0 && lane == 0) WMTP_TRACE_TILE(1, it);
         const TileMeta m = meta[stage];
         bool patched = false;
         if (CL && a.n_new > 0 && m.nvalid > 0) {
@@ -643,83 +745,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             }
         }
 
-        if (m.flags & kFirst) {
-            // ---- unit start: load this warp's Q rows, visibility masks, reset state -------
-            Lpre = m.L_tot - a.n_q;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
-                row_ok[r] = R < a.rows_total;
-                const int i = row_ok[r] ? R / a.G : 0;
-                vis[r] = step_visibility(a, m.b, i);
-                m_r[r] = -INFINITY;
-                l_r[r] = 0.f;
-            }
-#pragma unroll
-            for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-            if constexpr (QS) {
-                // every warp is past the previous unit's reads of these rows; each consumer thread
-                // widens quarter rows (32 dims) of the unit's Q into shared memory
-                if (!consumers_sync()) { alive = false; break; }
-                for (int w = threadIdx.x; w < NMT * 16 * 4; w += NWC * 32) {
-                    const int row = w >> 2, part = w & 3;
-                    const int R = m.rb * kRowsPerBlock + row;
-                    uint32_t h[16];
-                    if (R < a.rows_total) {
-                        const int i = R / a.G, g = R - (R / a.G) * a.G;
-                        const uint4* src = reinterpret_cast<const uint4*>(
-                            a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD + 32 * part);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint4 v = __ldg(src + k);
-                            h[4 * k] = bf16x2_to_f16x2(v.x);
-                            h[4 * k + 1] = bf16x2_to_f16x2(v.y);
-                            h[4 * k + 2] = bf16x2_to_f16x2(v.z);
-                            h[4 * k + 3] = bf16x2_to_f16x2(v.w);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) h[k] = 0u;
-                    }
-                    const uint32_t dst = smem_addr(smem + L::kQOff) + (uint32_t)(row * L::kQStride + 64 * part);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                                     :: "r"(dst + 16u * k), "r"(h[4 * k]), "r"(h[4 * k + 1]),
-                                        "r"(h[4 * k + 2]), "r"(h[4 * k + 3]) : "memory");
-                }
-                if (!consumers_sync()) { alive = false; break; }
-            } else {
-            const uint32_t* q32[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int R = m.rb * kRowsPerBlock + mt * 16 + gid + r * 8;
-                const int i = R / a.G, g = R - (R / a.G) * a.G;
-                q32[r] = reinterpret_cast<const uint32_t*>(
-                    a.q + (((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g) * kD);
-            }
-            if (KV8) {
-                // fp16 A-fragments with the k order of the fp8 K fragments: k slots (2 tig, +1)
-                // and (2 tig + 8, +9) of step ks hold dims 16 ks + 4 tig + (0, 1) and (2, 3)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int c = ks * 8 + 2 * tig;
-                    qa[ks][0] = row_ok[0] ? bf16x2_to_f16x2(__ldg(q32[0] + c)) : 0u;
-                    qa[ks][1] = row_ok[1] ? bf16x2_to_f16x2(__ldg(q32[1] + c)) : 0u;
-                    qa[ks][2] = row_ok[0] ? bf16x2_to_f16x2(__ldg(q32[0] + c + 1)) : 0u;
-                    qa[ks][3] = row_ok[1] ? bf16x2_to_f16x2(__ldg(q32[1] + c + 1)) : 0u;
-                }
-            } else {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int c = ks * 8 + tig;     // 32-bit word index of dims (16 ks + 2 tig)
-                    qa[ks][0] = row_ok[0] ? __ldg(q32[0] + c) : 0u;
-                    qa[ks][1] = row_ok[1] ? __ldg(q32[1] + c) : 0u;
-                    qa[ks][2] = row_ok[0] ? __ldg(q32[0] + c + 4) : 0u;
-                    qa[ks][3] = row_ok[1] ? __ldg(q32[1] + c + 4) : 0u;
-                }
-            }
-            }
+        if ((m.flags & kFirst) && !(CL && it == 0)) {
+            if (!unit_start(m)) { alive = false; break; }
         }
 
         if (warp == 0 && lane == 0 && (m.flags & kFirst)) WMTP_TRACE_AT(11);
@@ -904,7 +931,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         if (CL && patched) fence_proxy_async();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[stage]);
-        if (warp == 0 && lane == 0 && it < 8) WMTP_TRACE_AT(20 + (int)it);
+        if (warp == 0 && lane == 0) WMTP_TRACE_TILE(2, it);
 
         if (m.flags & kLast) {
             // ---- unit end: combine key groups, then write the result or a partial ----------
@@ -1052,14 +1079,17 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 
 // ---------------------------------------------------------------------------------------------
 // lse_merge_kernel: combines the split partials of units that span several CTAs, and writes
-// empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block), 128
+// empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block), 256
 // threads.  Partial s has weight 2^(lse_s - max_s lse_s); empty partials have lse = -inf and
-// weight 0.  The partials' LSEs are read by all threads in parallel; then each warp sums a
-// quarter of the partials with 16-byte loads and the four warp sums are combined per head dim.
+// weight 0.  The partials' LSEs are read by all threads in parallel; then each of the eight
+// warps sums every 8th partial with 16-byte loads, eight partials in flight per lane (the merge
+// is a chain of L2 round trips: a 128K-key verify unit spans ~150 CTAs), and the warp sums are
+// combined per head dim.
 constexpr int kMaxParts = 1024;
+constexpr int kMergeThreads = 256;
 
 template <int SRC>
-__global__ void __launch_bounds__(kD)
+__global__ void __launch_bounds__(kMergeThreads)
 lse_merge_kernel(const AttnArgs a, int P_launch) {
     pdl_launch_dependents();
     pdl_wait();
@@ -1070,10 +1100,11 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     const int b = u / (a.n_rb * a.Hkv);
     const int R = rb * kRowsPerBlock + rr;
     if (R >= a.rows_total) return;
+    constexpr int kWarps = kMergeThreads / 32;
 
     __shared__ long long s_info[3];     // T, unit start, unit tiles
     __shared__ float s_w[kMaxParts];
-    __shared__ float s_red[kD / 32];
+    __shared__ float s_red[kWarps];
     if (threadIdx.x == 0) {
         long long T = 0, start = 0;
         int nt_u = 0;
@@ -1089,10 +1120,10 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     const int nt_u = (int)s_info[2];
     const int i = R / a.G, g = R - (R / a.G) * a.G;
     const size_t orow = ((size_t)b * a.n_q + i) * a.Hq + (size_t)h * a.G + g;
-    const int d = threadIdx.x;
+    const int tid = threadIdx.x;
     if (nt_u == 0) {
-        a.out[orow * kD + d] = __float2bfloat16_rn(0.f);
-        if (a.lse != nullptr && d == 0) a.lse[orow] = -INFINITY;
+        if (tid < kD) a.out[orow * kD + tid] = __float2bfloat16_rn(0.f);
+        if (a.lse != nullptr && tid == 0) a.lse[orow] = -INFINITY;
         return;
     }
     const int peff = plan_ctas(T, P_launch, a.min_tiles_per_cta);
@@ -1102,64 +1133,61 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     const int np = c_hi - c_lo + 1;     // <= peff <= P_launch <= kMaxParts (host-checked)
     const float* lse_base = a.ws_lse + (size_t)(c_lo + u) * a.rows_blk + rr;
     float mx = -INFINITY;
-    for (int k = d; k < np; k += kD) {
+    for (int k = tid; k < np; k += kMergeThreads) {
         const float x = lse_base[(size_t)k * a.rows_blk];
         s_w[k] = x;
         mx = fmaxf(mx, x);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if ((d & 31) == 0) s_red[d >> 5] = mx;
+    if ((tid & 31) == 0) s_red[tid >> 5] = mx;
     __syncthreads();
     mx = s_red[0];
 #pragma unroll
-    for (int k = 1; k < kD / 32; ++k) mx = fmaxf(mx, s_red[k]);
-    for (int k = d; k < np; k += kD) s_w[k] = (mx == -INFINITY) ? 0.f : exp2f(s_w[k] - mx);
+    for (int k = 1; k < kWarps; ++k) mx = fmaxf(mx, s_red[k]);
+    for (int k = tid; k < np; k += kMergeThreads) s_w[k] = (mx == -INFINITY) ? 0.f : exp2f(s_w[k] - mx);
     __syncthreads();
-    // Each warp takes every 4th partial; lane l owns head dims [4l, 4l + 4) (one 16-byte load
-    // per partial, 512 contiguous bytes per warp), four partials in flight per step.
-    const int warp = d >> 5, lane = d & 31;
+    // Warp w takes partials w, w + 8, ...; lane l owns head dims [4l, 4l + 4) (one 16-byte load
+    // per partial, 512 contiguous bytes per warp), eight partials in flight.
+    const int warp = tid >> 5, lane = tid & 31;
     const float4* o_base = reinterpret_cast<const float4*>(
         a.ws_o + ((size_t)(c_lo + u) * a.rows_blk + rr) * kD) + lane;
     const size_t kSlotStride4 = (size_t)a.rows_blk * (kD / 4);
-    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
-    int k = warp;
-    for (; k + 12 < np; k += 16) {
-        const float4 x0 = o_base[(size_t)k * kSlotStride4];
-        const float4 x1 = o_base[(size_t)(k + 4) * kSlotStride4];
-        const float4 x2 = o_base[(size_t)(k + 8) * kSlotStride4];
-        const float4 x3 = o_base[(size_t)(k + 12) * kSlotStride4];
-        const float w0 = s_w[k], w1 = s_w[k + 4], w2 = s_w[k + 8], w3 = s_w[k + 12];
-        acc0.x += w0 * x0.x + w2 * x2.x; acc0.y += w0 * x0.y + w2 * x2.y;
-        acc0.z += w0 * x0.z + w2 * x2.z; acc0.w += w0 * x0.w + w2 * x2.w;
-        acc1.x += w1 * x1.x + w3 * x3.x; acc1.y += w1 * x1.y + w3 * x3.y;
-        acc1.z += w1 * x1.z + w3 * x3.z; acc1.w += w1 * x1.w + w3 * x3.w;
-        wsum += (w0 + w1) + (w2 + w3);
+    for (int k0 = warp; k0 < np; k0 += 8 * kWarps) {
+        float4 x[8];
+        float wv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int k = k0 + j * kWarps;
+            wv[j] = k < np ? s_w[k] : 0.f;
+            x[j] = k < np ? o_base[(size_t)k * kSlotStride4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            acc.x += wv[j] * x[j].x; acc.y += wv[j] * x[j].y; acc.z += wv[j] * x[j].z; acc.w += wv[j] * x[j].w;
+            wsum += wv[j];
+        }
     }
-    for (; k < np; k += 4) {
-        const float4 x0 = o_base[(size_t)k * kSlotStride4];
-        const float w0 = s_w[k];
-        acc0.x += w0 * x0.x; acc0.y += w0 * x0.y; acc0.z += w0 * x0.z; acc0.w += w0 * x0.w;
-        wsum += w0;
-    }
-    __shared__ float4 s_acc[kD / 32][32];
-    __shared__ float s_wsum[kD / 32];
-    s_acc[warp][lane] = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+    __shared__ float4 s_acc[kWarps][32];
+    __shared__ float s_wsum[kWarps];
+    s_acc[warp][lane] = acc;
     if (lane == 0) s_wsum[warp] = wsum;
     __syncthreads();
-    // thread d sums head dim d over the four warps
+    if (tid >= kD) return;
+    // thread d sums head dim d over the warps
     const float* s_flat = reinterpret_cast<const float*>(s_acc);
-    const int l4 = d >> 2, c4 = d & 3;
-    float acc = 0.f, wt = 0.f;
+    const int l4 = tid >> 2, c4 = tid & 3;
+    float accd = 0.f, wt = 0.f;
 #pragma unroll
-    for (int g = 0; g < kD / 32; ++g) {
-        acc += s_flat[(g * 32 + l4) * 4 + c4];
-        wt += s_wsum[g];
+    for (int w = 0; w < kWarps; ++w) {
+        accd += s_flat[(w * 32 + l4) * 4 + c4];
+        wt += s_wsum[w];
     }
-    const float res = wt > 0.f ? acc / wt : 0.f;
-    a.out[orow * kD + d] = __float2bfloat16_rn(res);
-    if (a.lse != nullptr && d == 0) a.lse[orow] = wt > 0.f ? (mx + log2f(wt)) * kLn2 : -INFINITY;
+    const float res = wt > 0.f ? accd / wt : 0.f;
+    a.out[orow * kD + tid] = __float2bfloat16_rn(res);
+    if (a.lse != nullptr && tid == 0) a.lse[orow] = wt > 0.f ? (mx + log2f(wt)) * kLn2 : -INFINITY;
 }
 
 }  // namespace wmtp

@@ -293,6 +293,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                     const uint32_t pq = it >> 1, sub = it & 1u, ks = pq % NK;
                     if (sub == 0u && !mbar_wait_bounded(&kempty[ks], ((pq / NK) & 1u) ^ 1u)) { alive = false; break; }
                     kmeta[2 * ks + sub] = m;
+                    WMTP_TRACE_TILE(0, it);
                     if (KV8) {
                         // fp8: the codes land as they are (QK^T reads E4M3 keys)
                         uint8_t* dst8 = smem + L::kKOff + ks * L::kKSlotBytes + sub * kTileBytes8;
@@ -318,6 +319,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                     const uint32_t vs = it % NV;
                     if (!mbar_wait_bounded(&vempty[vs], ((it / NV) & 1u) ^ 1u)) { alive = false; break; }
                     vmeta[vs] = m;
+                    WMTP_TRACE_TILE(1, it);
                     if (m.nvalid > 0) {
                         mbar_arrive_expect_tx(&v8full[vs], kTileBytes8);
                         tma_load_3d(smem + L::kVOff + vs * kTileBytes + kHalfBytes, &vmap, &v8full[vs], 0, ty, tz, pol);
@@ -361,6 +363,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             for (uint32_t pq = 0; pq < npairs && ok; ++pq) {
                 const uint32_t ks = pq % NK, sb = pq % NSB;
                 if (!mbar_wait_bounded(&kfull[ks], (pq / NK) & 1u)) break;
+                WMTP_TRACE_TILE(7, 2 * pq);
                 const bool has1 = 2 * pq + 1 < n;
                 TileMeta mt[2];
                 uint32_t qb[2] = {0u, 0u};
@@ -427,6 +430,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 tc::commit(&kempty[ks]);
                 tc::commit(&s_full[sb]);
                 mbar_arrive(&s_full[sb]);
+                WMTP_TRACE_TILE(3, 2 * pq);
                 if (mt[0].flags & kLast) tc::commit(&q_free[qb[0]]);
                 if (has1 && (mt[1].flags & kLast)) tc::commit(&q_free[qb[1]]);
             }
@@ -462,6 +466,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 }
                 tc::commit(&p_free[sb]);
                 tc::commit(&vempty[vs]);
+                WMTP_TRACE_TILE(5, t);
             }
             tc::commit(&mma_done[1]);
             mbar_wait_bounded(&mma_done[1], 0);
@@ -574,6 +579,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&vfull[vs]);
+            if (lane == 0 && (warp & 1) == 0) WMTP_TRACE_TILE(2, t);
         }
         // pair 0's last tile (n - 2) ended its unit: tile n - 1 starts one more unit
         if (pair == 0u && qok && n >= 2 && (n & 1u) == 0u && (last.flags & kLast) &&
@@ -755,6 +761,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[sb]);
+            if (lane == 0 && warp == gwarp0) WMTP_TRACE_TILE(4, it);
             // ---- unit end: combine both groups' (O, max, sum), write the rows ----------------
             if (m.flags & kLast) {
                 if (!mbar_wait_bounded(&p_free[sb], (it / kPB) & 1u)) { alive = false; break; }

@@ -102,6 +102,23 @@ int encode_rows_map(CUtensorMap* map, const void* base, long long rows, long lon
     return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
 }
 
+// Build-time option (measurement): the stream-K / cluster split kernels load a bf16 K or V tile
+// with one 4-D box, (64 dims, 64 rows, 2 halves, block), which lands as the two 64-dim halves
+// one after the other -- the layout of two 64 x 64 boxes -- with half the TMA instructions.
+int encode_rows_map4(CUtensorMap* map, const void* base, long long rows, long long n_blocks) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    int rc = encoder(&enc);
+    if (rc != WMTP_OK) return rc;
+    cuuint64_t dims[4] = {64, (cuuint64_t)rows, 2, (cuuint64_t)n_blocks};
+    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, 128, (cuuint64_t)rows * kD * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)kTileKeys, 2, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
+}
+
 // Q of a call, [B, n_q, Hq, 128] bf16, viewed per kv head as 4-D (dim, g, h, b * n_q + i) and
 // read in boxes of (64 dims, G heads, 1 kv head, n_q queries): one box lands as the unit's rows
 // i * G + g, 128 bytes each, 128-byte swizzled (the tcgen05 A-operand layout).
@@ -239,6 +256,16 @@ int set_smem_once(K kern, int bytes, bool (&done)[kMaxDevices]) {
 #ifndef WMTP_TC8_MIN_ROWS
 #define WMTP_TC8_MIN_ROWS 17
 #endif
+// fp8 tcgen05 rings (build-time for sweeps): K pair slots (16 KiB of codes each) and V slots
+// (16 KiB fp16 each, an even number).  A V slot stays busy from its TMA issue through the
+// landing, the widening and PV (~2.9 us at 1M keys), so the V ring needs ~6 slots to keep a tile
+// every ~0.5 us.
+#ifndef WMTP_TC8_NK
+#define WMTP_TC8_NK 3
+#endif
+#ifndef WMTP_TC8_NV
+#define WMTP_TC8_NV 6
+#endif
 enum class Kern { kSplit16, kSplit32, kSplit64, kTc, kSplit16Fp8, kSplit32Fp8, kSplit64Fp8, kTcFp8 };
 
 Kern select_kernel(const Shape& s, bool kv8) {
@@ -271,7 +298,7 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
     const int grid = sm_count * MINB;
     rc = launch(kern, dim3(grid), dim3((NMT * NKG + 1) * 32), Lay::kAlloc, st, km, vm, a);
     if (rc != WMTP_OK) return rc;
-    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
+    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kMergeThreads), 0, st, a, grid);
 }
 
 template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
@@ -288,7 +315,7 @@ int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q
     const int grid = sm_count;
     rc = launch(kern, dim3(grid), dim3(tc_threads<KV8>()), Lay::kAlloc, st, km, vm, qm, a);
     if (rc != WMTP_OK) return rc;
-    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kD), 0, st, a, grid);
+    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kMergeThreads), 0, st, a, grid);
 }
 
 template <int SRC>
@@ -302,7 +329,8 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
         case Kern::kSplit16Fp8: return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);
         case Kern::kSplit32Fp8: return launch_attn_t<SRC, 2, 2, 4, 2, true>(km, vm, a, sm_count, s, st);
         case Kern::kSplit64Fp8: return launch_attn_t<SRC, 4, 1, 4, 2, true>(km, vm, a, sm_count, s, st);
-        case Kern::kTcFp8: return launch_attn_tc_t<SRC, 4, 4, 2, true>(km, vm, a.q, a, sm_count, s, st);
+        case Kern::kTcFp8:
+            return launch_attn_tc_t<SRC, WMTP_TC8_NK, WMTP_TC8_NV, 2, true>(km, vm, a.q, a, sm_count, s, st);
     }
     return WMTP_ERR_ARG;
 }
@@ -463,6 +491,14 @@ int paged_call(const wmtp_bf16* q, const void* k_pool, const void* v_pool,
     a.max_pages = max_pages;
     a.num_pages = num_pages;
     CUtensorMap km, vm;
+#ifdef WMTP_TMA4D
+    const Kern kk = select_kernel(s, kv8);
+    if (!kv8 && kk != Kern::kTc) {
+        if ((rc = encode_rows_map4(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
+        if ((rc = encode_rows_map4(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
+        return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st, kv8);
+    }
+#endif
     if ((rc = encode_rows_map(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv, kv8)) != WMTP_OK) return rc;
     if ((rc = encode_rows_map(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv, kv8)) != WMTP_OK) return rc;
     return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st, kv8);
@@ -636,8 +672,18 @@ int window_call(const wmtp_bf16* q, void* ring_k, void* ring_v, int64_t* ring_le
         a.n_new = n_new;
     }
     CUtensorMap km, vm;
-    if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
-    if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
+#ifdef WMTP_TMA4D
+    const bool four_d = !kv8 && !((stream_k || s.units > 65535) && select_kernel(s, kv8) == Kern::kTc);
+#else
+    const bool four_d = false;
+#endif
+    if (four_d) {
+        if ((rc = encode_rows_map4(&km, ring_k, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
+        if ((rc = encode_rows_map4(&vm, ring_v, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
+    } else {
+        if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
+        if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
+    }
     if (stream_k || s.units > 65535)
         return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, st, kv8);
     // tiles of the longest key set: the sink's, the window's, one more where the window wraps

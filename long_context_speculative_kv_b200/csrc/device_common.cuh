@@ -37,16 +37,30 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 // Build-time timestamp trace for measurement (off unless WMTP_TRACE is defined): named points of
 // CTA (0, 0) record the global timer; read with wmtp_trace_read.
+// WMTP_TRACE_TILE(role, t) records tile t - kTraceT0 (of the first 32 tiles from kTraceT0) of one
+// role in slot 64 + 32 role + (t - kTraceT0).
 #ifdef WMTP_TRACE
-constexpr int kTraceSlots = 64;
+constexpr int kTraceSlots = 64 + 32 * 8;
+#ifndef WMTP_TRACE_T0
+#define WMTP_TRACE_T0 0
+#endif
+constexpr int kTraceT0 = WMTP_TRACE_T0;
 __device__ unsigned long long g_trace[kTraceSlots];
 #define WMTP_TRACE_AT(i)                                                            \
     do {                                                                            \
         if (blockIdx.x == 0 && blockIdx.y == 0 && (i) < kTraceSlots) g_trace[(i)] = global_ns(); \
     } while (0)
+#define WMTP_TRACE_TILE(role, t)                                                    \
+    do {                                                                            \
+        const int tt_ = (int)(t) - kTraceT0;                                        \
+        if (tt_ >= 0 && tt_ < 32) WMTP_TRACE_AT(64 + 32 * (role) + tt_);             \
+    } while (0)
 #else
 #define WMTP_TRACE_AT(i) \
     do {                 \
+    } while (0)
+#define WMTP_TRACE_TILE(role, t) \
+    do {                         \
     } while (0)
 #endif
 
@@ -115,6 +129,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 4-D tiled load with an L2 cache hint (no multicast).
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, int z, int w, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w),
+          "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -152,16 +177,18 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank
     return r;
 }
 
+// (Reads of partials the cluster barrier has published: no ordering constraints of their own, so
+// the compiler may batch them.)
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
 }
 
 __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
     float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+    asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
     return v;
 }
 
