@@ -551,16 +551,10 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     tma_load_3d(st + kTileBytes8, &vmap, &full_bar[stage], 0, ty, tz, pol);
                 } else if (m.nvalid > 0) {
                     mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-#ifdef WMTP_TMA4D
-                    // one box per tensor: (64 dims, 64 rows, 2 halves) lands as [half][row][64]
-                    tma_load_4d_hint(st, &kmap, &full_bar[stage], 0, ty, 0, tz, pol);
-                    tma_load_4d_hint(st + kTileBytes, &vmap, &full_bar[stage], 0, ty, 0, tz, pol);
-#else
                     tma_load_3d(st, &kmap, &full_bar[stage], 0, ty, tz, pol);
                     tma_load_3d(st + kHalfBytes, &kmap, &full_bar[stage], 64, ty, tz, pol);
                     tma_load_3d(st + kTileBytes, &vmap, &full_bar[stage], 0, ty, tz, pol);
                     tma_load_3d(st + kTileBytes + kHalfBytes, &vmap, &full_bar[stage], 64, ty, tz, pol);
-#endif
                 } else {
                     mbar_arrive(&full_bar[stage]);
                 }

@@ -377,6 +377,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 }
                 if (!ok) break;
                 if (!mbar_wait_bounded(&s_free[sb], ((pq / NSB) & 1u) ^ 1u)) break;
+                WMTP_TRACE_TILE(6, 2 * pq);
                 smeta[2 * sb] = mt[0];
                 if (has1) smeta[2 * sb + 1] = mt[1];
                 tc::fence_after_sync();

@@ -102,23 +102,6 @@ int encode_rows_map(CUtensorMap* map, const void* base, long long rows, long lon
     return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
 }
 
-// Build-time option (measurement): the stream-K / cluster split kernels load a bf16 K or V tile
-// with one 4-D box, (64 dims, 64 rows, 2 halves, block), which lands as the two 64-dim halves
-// one after the other -- the layout of two 64 x 64 boxes -- with half the TMA instructions.
-int encode_rows_map4(CUtensorMap* map, const void* base, long long rows, long long n_blocks) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc;
-    int rc = encoder(&enc);
-    if (rc != WMTP_OK) return rc;
-    cuuint64_t dims[4] = {64, (cuuint64_t)rows, 2, (cuuint64_t)n_blocks};
-    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, 128, (cuuint64_t)rows * kD * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)kTileKeys, 2, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? WMTP_OK : WMTP_ERR_CUDA;
-}
-
 // Q of a call, [B, n_q, Hq, 128] bf16, viewed per kv head as 4-D (dim, g, h, b * n_q + i) and
 // read in boxes of (64 dims, G heads, 1 kv head, n_q queries): one box lands as the unit's rows
 // i * G + g, 128 bytes each, 128-byte swizzled (the tcgen05 A-operand layout).
@@ -372,15 +355,18 @@ int cluster_capacity(K kern, int smem, int threads, int cs, int (&cache)[kMaxDev
 }
 
 // Build-time options for measurement sweeps: the largest cluster size, and the stage count /
-// CTAs per SM of the layout for units of at most 16 rows.
+// CTAs per SM of the layout for units of at most 16 rows.  Two stages and two CTAs per SM
+// (94 KB of shared memory each) rather than the stream-K kernel's four stages and one CTA: the
+// smaller CTAs let eight 16-CTA clusters be resident at once (the NoPE workload's 8 units; at
+// 160 KB per CTA only clusters of 8 fit), 64 MiB window call 27.7 -> 20.2 us.
 #ifndef WMTP_CL_MAX
 #define WMTP_CL_MAX 16
 #endif
 #ifndef WMTP_CL16_NSTAGE
-#define WMTP_CL16_NSTAGE 4
+#define WMTP_CL16_NSTAGE 2
 #endif
 #ifndef WMTP_CL16_MINB
-#define WMTP_CL16_MINB 1
+#define WMTP_CL16_MINB 2
 #endif
 
 template <int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
@@ -491,14 +477,6 @@ int paged_call(const wmtp_bf16* q, const void* k_pool, const void* v_pool,
     a.max_pages = max_pages;
     a.num_pages = num_pages;
     CUtensorMap km, vm;
-#ifdef WMTP_TMA4D
-    const Kern kk = select_kernel(s, kv8);
-    if (!kv8 && kk != Kern::kTc) {
-        if ((rc = encode_rows_map4(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
-        if ((rc = encode_rows_map4(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv)) != WMTP_OK) return rc;
-        return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st, kv8);
-    }
-#endif
     if ((rc = encode_rows_map(&km, k_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv, kv8)) != WMTP_OK) return rc;
     if ((rc = encode_rows_map(&vm, v_pool, WMTP_PAGE_SIZE, (long long)num_pages * Hkv, kv8)) != WMTP_OK) return rc;
     return launch_attn<kSrcPaged>(km, vm, a, dev.sm_count, s, st, kv8);
@@ -672,18 +650,8 @@ int window_call(const wmtp_bf16* q, void* ring_k, void* ring_v, int64_t* ring_le
         a.n_new = n_new;
     }
     CUtensorMap km, vm;
-#ifdef WMTP_TMA4D
-    const bool four_d = !kv8 && !((stream_k || s.units > 65535) && select_kernel(s, kv8) == Kern::kTc);
-#else
-    const bool four_d = false;
-#endif
-    if (four_d) {
-        if ((rc = encode_rows_map4(&km, ring_k, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
-        if ((rc = encode_rows_map4(&vm, ring_v, capacity, (long long)B * Hkv)) != WMTP_OK) return rc;
-    } else {
-        if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
-        if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
-    }
+    if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
+    if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
     if (stream_k || s.units > 65535)
         return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, st, kv8);
     // tiles of the longest key set: the sink's, the window's, one more where the window wraps
