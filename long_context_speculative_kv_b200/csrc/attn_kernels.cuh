@@ -316,6 +316,12 @@ struct SmemLayout {
     static constexpr int kPlanBytes = 2 * kMaxBatch * 4;            // tiles per request, length
     static constexpr int kTotal = kPlanOff + kPlanBytes;
     static constexpr int kAlloc = kTotal + 1024;                     // slack for base alignment
+    // cluster window mode: the CTA's (o, lse) partial of its unit lives in the stage space once
+    // the pipeline has drained: [NMT * 16 rows][128] fp32 normalised outputs, then the rows'
+    // base-2 LSEs
+    static constexpr int kPartOff = 0;
+    static constexpr int kPartLseOff = NMT * 16 * kD * 4;
+    static_assert(kPartLseOff + NMT * 16 * 4 <= kStagesBytes, "partial fits the stage space");
 };
 
 // Swizzled shared address of 16-byte chunk `chunk` (0..15) of key row `row` in a K/V tile
@@ -330,79 +336,53 @@ __device__ __forceinline__ uint32_t tile8_chunk_addr(uint32_t base, int row, int
 }
 
 // ---------------------------------------------------------------------------------------------
-// Cluster window mode, end of the kernel.  Row rr of the unit belongs to CTA rr % size (its local
-// row j = rr / size).  After a first cluster barrier (every CTA is past its tiles, so the stage
-// space is free everywhere) each consumer warp stores its key group's normalised (o, lse) partial
-// of each of its rows into the owning CTA's receive area -- the stage space, slots [j][sender]
-// with sender = rank * NKG + key group -- as remote shared-memory stores; after a second cluster
-// barrier (every store has landed) each CTA merges its own rows from local shared memory.  No
-// CTA reads another CTA's shared memory, so none has to wait for its siblings before leaving.
+// Cluster window mode, end of the kernel: merges the cluster's per-CTA partials of its unit
+// through distributed shared memory.  Every thread of the CTA calls it exactly once.  CTA `me`
+// takes the unit's rows me, me + size, ...; one warp per row: lane k reads rank k's LSE (ranks
+// without tiles hold no partial), then lane l sums head dims 4 l .. 4 l + 3 over the ranks with
+// one 16-byte remote load per rank.  The second cluster barrier keeps every CTA's shared memory
+// alive until its siblings have read it.
 template <int NMT, int NKG, int NSTAGE, bool KV8, bool QS>
-struct ClusterRecv {
+__device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* smem,
+                                                   const RingUnitWalker& wk, int nt, int warp,
+                                                   int lane) {
     using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
-    static constexpr int kMaxSlots = NMT * 16 * NKG;            // ceil(rows / size) * size * NKG <= this
-    static constexpr int kOOff = 0;                             // [slot][128] fp32
-    static constexpr int kLseOff = kMaxSlots * kD * 4;          // [slot] fp32 (base-2 LSE)
-    static_assert(kLseOff + kMaxSlots * 4 <= L::kMergeMLOff, "receive area fits the stage and merge space");
-};
-
-// Pushes one row's partial (this thread's head dims of it) to the owning CTA.
-template <bool KV8>
-__device__ __forceinline__ void cluster_push_row(uint8_t* smem, int recv_o, int recv_lse, int slot,
-                                                 uint32_t owner, const float (&o)[16][4], int r,
-                                                 float inv, float lse2, int tig) {
-    const uint32_t ob = map_shared_rank(smem_addr(smem + recv_o) + 4u * (uint32_t)(slot * kD), owner);
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const int d = KV8 ? 16 * (n >> 1) + 4 * tig + 2 * (n & 1) : 8 * n + 2 * tig;
-        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};"
-                     :: "r"(ob + 4u * (uint32_t)d), "f"(o[n][2 * r] * inv), "f"(o[n][2 * r + 1] * inv)
-                     : "memory");
-    }
-    if (tig == 0) {
-        const uint32_t lb = map_shared_rank(smem_addr(smem + recv_lse) + 4u * (uint32_t)slot, owner);
-        asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(lb), "f"(lse2) : "memory");
-    }
-}
-
-// Merges this CTA's rows of the unit from its receive area (after the second cluster barrier).
-template <int NMT, int NKG, int NSTAGE, bool KV8, bool QS>
-__device__ __forceinline__ void cluster_merge_local(const AttnArgs& a, uint8_t* smem, const RingUnitWalker& wk,
-                                                    int nt, int warp, int lane) {
-    using R = ClusterRecv<NMT, NKG, NSTAGE, KV8, QS>;
     constexpr int kWarps = NMT * NKG + 1;
+    cluster_sync_all();
+    if (warp == 0 && lane == 0) WMTP_TRACE_AT(29);
     const int cs = (int)gridDim.x, me = (int)blockIdx.x;
-    const int nk = cs * NKG;                                    // senders per row (<= 64)
     const int rows_u = min(kRowsPerBlock, a.rows_total - wk.rb * kRowsPerBlock);
-    const float* ro = reinterpret_cast<const float*>(smem + R::kOOff);
-    const float* rl = reinterpret_cast<const float*>(smem + R::kLseOff);
-    // a sender slot holds a partial only if its rank had tiles
-    auto has = [&](int k) -> bool {
-        const long long rk = k / NKG;
-        return k < nk && (rk + 1) * nt / cs > rk * nt / cs;
-    };
-    for (int j = warp; me + j * cs < rows_u; j += kWarps) {
-        const int rr = me + j * cs;
-        const int s0 = j * nk;
-        const float x0 = has(lane) ? rl[s0 + lane] : -INFINITY;
-        const float x1 = has(lane + 32) ? rl[s0 + lane + 32] : -INFINITY;
-        float mx = fmaxf(x0, x1);
+    const uint32_t part = smem_addr(smem + L::kPartOff);
+    const uint32_t plse = smem_addr(smem + L::kPartLseOff);
+    const bool has = lane < cs && (long long)(lane + 1) * nt / cs > (long long)lane * nt / cs;
+    for (int rr = me + warp * cs; rr < rows_u; rr += kWarps * cs) {
+        float x = -INFINITY;
+        if (has) x = ld_dsmem_f32(map_shared_rank(plse + 4u * rr, lane));
+        float mx = x;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float w0 = mx != -INFINITY && x0 != -INFINITY ? exp2f(x0 - mx) : 0.f;
-        const float w1 = mx != -INFINITY && x1 != -INFINITY ? exp2f(x1 - mx) : 0.f;
+        const float w = (has && mx != -INFINITY) ? exp2f(x - mx) : 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float wsum = 0.f;
-        for (int k = 0; k < nk; ++k) {
-            const float wk_ = __shfl_sync(0xffffffffu, k < 32 ? w0 : w1, k & 31);
-            if (wk_ > 0.f) {
-                const float4 v = *reinterpret_cast<const float4*>(ro + (size_t)(s0 + k) * kD + 4 * lane);
-                acc.x += wk_ * v.x; acc.y += wk_ * v.y; acc.z += wk_ * v.z; acc.w += wk_ * v.w;
-                wsum += wk_;
+        const uint32_t po = part + 4u * (uint32_t)(rr * kD + 4 * lane);
+        // eight ranks' loads in flight at a time (a load waited on before the next is issued
+        // would cost one distributed-shared-memory round trip per rank)
+        for (int k0 = 0; k0 < cs; k0 += 8) {
+            float4 v[8];
+            float wv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                wv[j] = (k0 + j < cs) ? __shfl_sync(0xffffffffu, w, k0 + j) : 0.f;
+                v[j] = wv[j] > 0.f ? ld_dsmem_v4(map_shared_rank(po, (uint32_t)(k0 + j))) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                acc.x += wv[j] * v[j].x; acc.y += wv[j] * v[j].y; acc.z += wv[j] * v[j].z; acc.w += wv[j] * v[j].w;
+                wsum += wv[j];
             }
         }
-        const int Rg = wk.rb * kRowsPerBlock + rr;
-        const int i = Rg / a.G, g = Rg - (Rg / a.G) * a.G;
+        const int R = wk.rb * kRowsPerBlock + rr;
+        const int i = R / a.G, g = R - (R / a.G) * a.G;
         const size_t orow = ((size_t)wk.b * a.n_q + i) * a.Hq + (size_t)wk.h * a.G + g;
         const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
         uint2 pk;
@@ -411,6 +391,9 @@ __device__ __forceinline__ void cluster_merge_local(const AttnArgs& a, uint8_t* 
         *reinterpret_cast<uint2*>(a.out + orow * kD + 4 * lane) = pk;
         if (a.lse != nullptr && lane == 0) a.lse[orow] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
     }
+    if (warp == 0 && lane == 0) WMTP_TRACE_AT(30);
+    __syncwarp();
+    cluster_sync_all();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -546,7 +529,6 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     if (warp == NWC) {
         // =========================== producer warp =========================================
         if (lane == 0 && t_begin < t_end) {
-            WMTP_TRACE_AT(40);
             const uint64_t pol = l2_evict_first_policy();
             TileWalker<SRC> walk;
             if (!CL) walk.init(a, plan_tiles);
@@ -558,7 +540,6 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     s_walk.describe(a, (int)t, (int)t_begin, (int)t_end, m, ty, tz);
                 else
                     walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
-                if (it == 0) WMTP_TRACE_AT(41);
                 const int stage = (int)(it % NSTAGE);
                 const uint32_t phase = (it / NSTAGE) & 1u;
                 if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) break;
@@ -570,9 +551,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     tma_load_3d(st + kTileBytes8, &vmap, &full_bar[stage], 0, ty, tz, pol);
                 } else if (m.nvalid > 0) {
                     mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-                    if (it == 0) WMTP_TRACE_AT(42);
                     tma_load_3d(st, &kmap, &full_bar[stage], 0, ty, tz, pol);
-                    if (it == 0) WMTP_TRACE_AT(43);
                     tma_load_3d(st + kHalfBytes, &kmap, &full_bar[stage], 64, ty, tz, pol);
                     tma_load_3d(st + kTileBytes, &vmap, &full_bar[stage], 0, ty, tz, pol);
                     tma_load_3d(st + kTileBytes + kHalfBytes, &vmap, &full_bar[stage], 64, ty, tz, pol);
@@ -590,10 +569,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         }
         if (CL) {
             __syncwarp();
-            cluster_sync_all();                 // every CTA past its tiles
-            __syncwarp();
-            cluster_sync_all();                 // every partial pushed
-            cluster_merge_local<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
+            cluster_merge_rows<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
         }
         return;
     }
@@ -625,7 +601,6 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     uint32_t it = 0;
     uint32_t sync_phase = 0;
     bool alive = true;
-    bool have_part = false;            // cluster mode: this warp holds its key group's partial
     // Bounded rendezvous of the consumer warps (an mbarrier, so a sibling that gave up on a
     // timed-out wait cannot leave the others blocked for ever).
     auto consumers_sync = [&]() -> bool {
@@ -959,9 +934,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 1);
                 l_r[r] += __shfl_xor_sync(0xffffffffu, l_r[r], 2);
             }
-            if (CL) {
-                have_part = true;               // pushed after the loop (cluster window mode)
-            } else if (QS && NKG > 1) {
+            if (QS && NKG > 1) {
                 // one m-tile at a time through the shared Q rows' space, once every warp is past
                 // its last reads of them
                 if (!consumers_sync()) { alive = false; break; }
@@ -1049,7 +1022,11 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
                 if (!consumers_sync()) { alive = false; break; }
             }
-            if (!CL && kg == 0) {
+            if (CL && NKG == 1) {
+                // every consumer warp is past its last reads of the stage space the partial takes
+                if (!consumers_sync()) { alive = false; break; }
+            }
+            if (kg == 0) {
                 const int slot = (int)blockIdx.x + m.unit;
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -1059,7 +1036,14 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     const float l = l_r[r];
                     const float inv = l > 0.f ? a.v_scale / l : 0.f;
                     const float lse2 = l > 0.f ? m_r[r] + __log2f(l) : -INFINITY;
-                    if (m.flags & kWhole) {
+                    if (CL) {
+                        float* po = reinterpret_cast<float*>(smem + L::kPartOff) + (size_t)rr * kD;
+#pragma unroll
+                        for (int n = 0; n < 16; ++n)
+                            *reinterpret_cast<float2*>(po + out_dim(n, tig)) =
+                                make_float2(o[n][2 * r] * inv, o[n][2 * r + 1] * inv);
+                        if (tig == 0) reinterpret_cast<float*>(smem + L::kPartLseOff)[rr] = lse2;
+                    } else if (m.flags & kWhole) {
                         const int i = R / a.G, g = R - (R / a.G) * a.G;
                         const size_t orow = ((size_t)m.b * a.n_q + i) * a.Hq + (size_t)m.h * a.G + g;
                         uint32_t* op = reinterpret_cast<uint32_t*>(a.out + orow * kD);
@@ -1081,28 +1065,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     if (warp == 0 && lane == 0) WMTP_TRACE_AT(28);
     if (CL) {
-        using RC = ClusterRecv<NMT, NKG, NSTAGE, KV8, QS>;
         __syncwarp();
-        cluster_sync_all();                     // every CTA past its tiles: receive areas free
-        if (warp == 0 && lane == 0) WMTP_TRACE_AT(29);
-        if (have_part) {
-            const int cs = (int)gridDim.x;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                if (!row_ok[r]) continue;
-                const int rr = mt * 16 + gid + 8 * r;
-                const float l = l_r[r];
-                const float inv = l > 0.f ? a.v_scale / l : 0.f;
-                const float lse2 = l > 0.f ? m_r[r] + __log2f(l) : -INFINITY;
-                const int slot = (rr / cs) * cs * NKG + (int)blockIdx.x * NKG + kg;
-                cluster_push_row<KV8>(smem, RC::kOOff, RC::kLseOff, slot, (uint32_t)(rr % cs), o, r, inv,
-                                      lse2, tig);
-            }
-        }
-        __syncwarp();
-        cluster_sync_all();                     // every partial has landed
-        if (warp == 0 && lane == 0) WMTP_TRACE_AT(30);
-        cluster_merge_local<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
+        cluster_merge_rows<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);
         if (warp == 0 && lane == 0) WMTP_TRACE_AT(31);
     }
 }

@@ -611,6 +611,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             const uint32_t scol = sq * 128u + 64u * grp;     // this tile's 64 score columns
             const uint32_t sb = it % kPB;                    // P buffer
             if (!mbar_wait_bounded(&s_full[sq], ((it >> 1) / NSB) & 1u)) { alive = false; break; }
+            if (lane == 0 && warp == gwarp0) WMTP_TRACE_TILE(8, it);
             tc::fence_after_sync();
             const TileMeta m = smeta[2 * sq + grp];
             if (m.unit != my_unit) {
@@ -637,6 +638,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             tc::ld_16x32bx2_x16<32>(tmem + lane_base + scol, sr);
             tc::ld_16x32bx2_x16<32>(tmem + lane_base + scol + 16u, sr + 16);
             tc::wait_ld();
+            if (lane == 0 && warp == gwarp0) WMTP_TRACE_TILE(9, it);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[sq]);
@@ -701,6 +703,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                 }
             }
             l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            if (lane == 0 && warp == gwarp0) WMTP_TRACE_TILE(10, it);
             // ---- P to shared memory (its buffer is free once PV of tile it - NSB is done) -----
             if (it >= (uint32_t)kPB && !mbar_wait_bounded(&p_free[sb], ((it / kPB) & 1u) ^ 1u)) {
                 alive = false;
@@ -715,6 +718,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 }
             }
+            if (lane == 0 && warp == gwarp0) WMTP_TRACE_TILE(11, it);
             // V rows past the valid keys may hold anything (NaN tails): zero them before PV
             if (m.nvalid > 0 && m.nvalid < kTileKeys) {
                 const uint32_t vs = it % NV;

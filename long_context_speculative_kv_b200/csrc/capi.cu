@@ -259,10 +259,17 @@ Kern select_kernel(const Shape& s, bool kv8) {
     return kv8 ? Kern::kSplit64Fp8 : Kern::kSplit64;
 }
 
+// Build-time option for measurement sweeps: 32-row units on one CTA per SM with four stages
+// (half the split partials per unit) instead of two CTAs with two stages.
+#ifndef WMTP_SPLIT32_ONE_CTA
+#define WMTP_SPLIT32_ONE_CTA 0
+#endif
+
 // CTAs per SM of each kernel (the grid is sm_count times this).
 int ctas_per_sm(Kern k) {
     switch (k) {
         case Kern::kSplit16: return 1;
+        case Kern::kSplit32: return WMTP_SPLIT32_ONE_CTA ? 1 : 2;
         case Kern::kSplit16Fp8: return 3;
         case Kern::kTc: case Kern::kTcFp8: return 1;
         default: return 2;
@@ -306,7 +313,12 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
                 const Shape& s, cudaStream_t st, bool kv8 = false) {
     switch (select_kernel(s, kv8)) {
         case Kern::kSplit16: return launch_attn_t<SRC, 1, 4, 4, 1>(km, vm, a, sm_count, s, st);
-        case Kern::kSplit32: return launch_attn_t<SRC, 2, 2, 2, 2>(km, vm, a, sm_count, s, st);
+        case Kern::kSplit32:
+#if WMTP_SPLIT32_ONE_CTA
+            return launch_attn_t<SRC, 2, 2, 4, 1>(km, vm, a, sm_count, s, st);
+#else
+            return launch_attn_t<SRC, 2, 2, 2, 2>(km, vm, a, sm_count, s, st);
+#endif
         case Kern::kSplit64: return launch_attn_t<SRC, 4, 1, 2, 2>(km, vm, a, sm_count, s, st);
         case Kern::kTc: return launch_attn_tc_t<SRC, 3, 3, 2>(km, vm, a.q, a, sm_count, s, st);
         case Kern::kSplit16Fp8: return launch_attn_t<SRC, 1, 4, 2, 3, true, true>(km, vm, a, sm_count, s, st);

@@ -40,7 +40,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 // WMTP_TRACE_TILE(role, t) records tile t - kTraceT0 (of the first 32 tiles from kTraceT0) of one
 // role in slot 64 + 32 role + (t - kTraceT0).
 #ifdef WMTP_TRACE
-constexpr int kTraceSlots = 64 + 32 * 8;
+constexpr int kTraceSlots = 64 + 32 * 12;
 #ifndef WMTP_TRACE_T0
 #define WMTP_TRACE_T0 0
 #endif
