@@ -449,12 +449,14 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) WMTP_TRACE_AT(0);
-    pdl_launch_dependents();
     if (warp == NWC && lane == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
+    // the successor may launch once this kernel's predecessor is done (so it may read, before
+    // its own wait, inputs this kernel does not write: the LSE merge reads the lengths early)
     pdl_wait();
+    pdl_launch_dependents();
     if (threadIdx.x == 0) WMTP_TRACE_AT(1);
 
     __shared__ RingUnitWalker s_walk;          // cluster mode: this CTA's unit
@@ -1073,20 +1075,26 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 
 // ---------------------------------------------------------------------------------------------
 // lse_merge_kernel: combines the split partials of units that span several CTAs, and writes
-// empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block), 256
-// threads.  Partial s has weight 2^(lse_s - max_s lse_s); empty partials have lse = -inf and
-// weight 0.  The partials' LSEs are read by all threads in parallel; then each of the eight
-// warps sums every 8th partial with 16-byte loads, eight partials in flight per lane (the merge
-// is a chain of L2 round trips: a 128K-key verify unit spans ~150 CTAs), and the warp sums are
-// combined per head dim.
+// empty units (no keys at all) as out = 0, lse = -inf.  Grid (units, rows per block, C head-dim
+// chunks of 128 / C dims), 256 threads.  Partial s has weight 2^(lse_s - M) with M the largest
+// partial LSE; empty partials have lse = -inf and weight 0.
+// The plan (which CTAs hold the unit's partials) needs only the request lengths, which the
+// attention kernel before this one does not write and which were final before it let this kernel
+// launch (it triggers after its own wait), so it is computed before this kernel's wait.  After the
+// wait, thread t takes partials t / F, t / F + 256 / F, ... (F = 32 / C float4 per partial chunk)
+// and float4 t % F of each, issues the LSE and 16-byte partial loads of kMergeBatch partials at
+// once and folds them into a running (max, sum, O); the threads' states are combined per head dim
+// in shared memory.  The host picks C so that one round of loads covers the expected partials (a
+// 128K-key verify unit has ~150: one L2 round trip).
 constexpr int kMaxParts = 1024;
 constexpr int kMergeThreads = 256;
+constexpr int kMergeBatch = 6;
 
 template <int SRC>
 __global__ void __launch_bounds__(kMergeThreads)
 lse_merge_kernel(const AttnArgs a, int P_launch) {
     pdl_launch_dependents();
-    pdl_wait();
+    if (threadIdx.x == 0) WMTP_TRACE_AT(48);
     const int u = blockIdx.x;
     const int rr = blockIdx.y;
     const int rb = u % a.n_rb;
@@ -1094,11 +1102,8 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
     const int b = u / (a.n_rb * a.Hkv);
     const int R = rb * kRowsPerBlock + rr;
     if (R >= a.rows_total) return;
-    constexpr int kWarps = kMergeThreads / 32;
 
-    __shared__ long long s_info[3];     // T, unit start, unit tiles
-    __shared__ float s_w[kMaxParts];
-    __shared__ float s_red[kWarps];
+    __shared__ int s_info[3];           // unit tiles, first and last CTA of the unit
     if (threadIdx.x == 0) {
         long long T = 0, start = 0;
         int nt_u = 0;
@@ -1107,81 +1112,89 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
             if (bb == b) { start = T + (long long)(h * a.n_rb + rb) * nt; nt_u = nt; }
             T += (long long)nt * a.Hkv * a.n_rb;
         }
-        s_info[0] = T; s_info[1] = start; s_info[2] = nt_u;
+        s_info[0] = nt_u;
+        if (nt_u > 0) {
+            const int peff = plan_ctas(T, P_launch, a.min_tiles_per_cta);
+            s_info[1] = cta_of_tile(start, T, peff);
+            s_info[2] = cta_of_tile(start + nt_u - 1, T, peff);
+        }
     }
     __syncthreads();
-    const long long T = s_info[0], start = s_info[1];
-    const int nt_u = (int)s_info[2];
+    const int nt_u = s_info[0];
     const int i = R / a.G, g = R - (R / a.G) * a.G;
     const size_t orow = ((size_t)b * a.n_q + i) * a.Hq + (size_t)h * a.G + g;
     const int tid = threadIdx.x;
+    const int C = gridDim.z, F = (kD / 4) / C, dims = kD / C, d_lo = blockIdx.z * dims;
+    pdl_wait();
+    if (threadIdx.x == 0) WMTP_TRACE_AT(49);
     if (nt_u == 0) {
-        if (tid < kD) a.out[orow * kD + tid] = __float2bfloat16_rn(0.f);
-        if (a.lse != nullptr && tid == 0) a.lse[orow] = -INFINITY;
+        if (tid < dims) a.out[orow * kD + d_lo + tid] = __float2bfloat16_rn(0.f);
+        if (a.lse != nullptr && tid == 0 && blockIdx.z == 0) a.lse[orow] = -INFINITY;
         return;
     }
-    const int peff = plan_ctas(T, P_launch, a.min_tiles_per_cta);
-    const int c_lo = cta_of_tile(start, T, peff);
-    const int c_hi = cta_of_tile(start + nt_u - 1, T, peff);
+    const int c_lo = s_info[1], c_hi = s_info[2];
     if (c_lo == c_hi) return;           // finished inside one CTA
     const int np = c_hi - c_lo + 1;     // <= peff <= P_launch <= kMaxParts (host-checked)
+    const int lanes = kMergeThreads / F;          // partials per load step
+    const int qk = tid / F, f4 = tid - qk * F;
     const float* lse_base = a.ws_lse + (size_t)(c_lo + u) * a.rows_blk + rr;
-    float mx = -INFINITY;
-    for (int k = tid; k < np; k += kMergeThreads) {
-        const float x = lse_base[(size_t)k * a.rows_blk];
-        s_w[k] = x;
-        mx = fmaxf(mx, x);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    if ((tid & 31) == 0) s_red[tid >> 5] = mx;
-    __syncthreads();
-    mx = s_red[0];
-#pragma unroll
-    for (int k = 1; k < kWarps; ++k) mx = fmaxf(mx, s_red[k]);
-    for (int k = tid; k < np; k += kMergeThreads) s_w[k] = (mx == -INFINITY) ? 0.f : exp2f(s_w[k] - mx);
-    __syncthreads();
-    // Warp w takes partials w, w + 8, ...; lane l owns head dims [4l, 4l + 4) (one 16-byte load
-    // per partial, 512 contiguous bytes per warp), eight partials in flight.
-    const int warp = tid >> 5, lane = tid & 31;
     const float4* o_base = reinterpret_cast<const float4*>(
-        a.ws_o + ((size_t)(c_lo + u) * a.rows_blk + rr) * kD) + lane;
+        a.ws_o + ((size_t)(c_lo + u) * a.rows_blk + rr) * kD + d_lo) + f4;
     const size_t kSlotStride4 = (size_t)a.rows_blk * (kD / 4);
+    float m_t = -INFINITY, s_t = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float wsum = 0.f;
-    for (int k0 = warp; k0 < np; k0 += 8 * kWarps) {
-        float4 x[8];
-        float wv[8];
+    for (int k0 = qk; k0 < np; k0 += kMergeBatch * lanes) {
+        float lv[kMergeBatch];
+        float4 x[kMergeBatch];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int k = k0 + j * kWarps;
-            wv[j] = k < np ? s_w[k] : 0.f;
-            x[j] = k < np ? o_base[(size_t)k * kSlotStride4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < kMergeBatch; ++j) {
+            const int k = k0 + j * lanes;
+            lv[j] = k < np ? __ldcg(lse_base + (size_t)k * a.rows_blk) : -INFINITY;
+            x[j] = k < np ? __ldcg(o_base + (size_t)k * kSlotStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        float mb = lv[0];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            acc.x += wv[j] * x[j].x; acc.y += wv[j] * x[j].y; acc.z += wv[j] * x[j].z; acc.w += wv[j] * x[j].w;
-            wsum += wv[j];
+        for (int j = 1; j < kMergeBatch; ++j) mb = fmaxf(mb, lv[j]);
+        if (mb > m_t) {
+            const float f = (m_t == -INFINITY) ? 0.f : exp2f(m_t - mb);
+            acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+            s_t *= f;
+            m_t = mb;
+        }
+        if (m_t == -INFINITY) continue;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) {
+            const float w = (lv[j] == -INFINITY) ? 0.f : exp2f(lv[j] - m_t);
+            acc.x += w * x[j].x; acc.y += w * x[j].y; acc.z += w * x[j].z; acc.w += w * x[j].w;
+            s_t += w;
         }
     }
-    __shared__ float4 s_acc[kWarps][32];
-    __shared__ float s_wsum[kWarps];
-    s_acc[warp][lane] = acc;
-    if (lane == 0) s_wsum[warp] = wsum;
+    if (threadIdx.x == 0) WMTP_TRACE_AT(50);
+    __shared__ float4 s_acc[kMergeThreads];
+    __shared__ float s_m[kMergeThreads], s_s[kMergeThreads];
+    s_acc[tid] = acc;
+    s_m[tid] = m_t;
+    s_s[tid] = s_t;
     __syncthreads();
-    if (tid >= kD) return;
-    // thread d sums head dim d over the warps
-    const float* s_flat = reinterpret_cast<const float*>(s_acc);
-    const int l4 = tid >> 2, c4 = tid & 3;
+    if (tid >= dims) return;
+    // thread d combines head dim d_lo + d over the partial lanes
+    const int fd = tid >> 2, cd = tid & 3;
+    float M = -INFINITY;
+    for (int q = 0; q < lanes; ++q) M = fmaxf(M, s_m[q * F + fd]);
     float accd = 0.f, wt = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        accd += s_flat[(w * 32 + l4) * 4 + c4];
-        wt += s_wsum[w];
+    if (M != -INFINITY) {
+        for (int q = 0; q < lanes; ++q) {
+            const float mq = s_m[q * F + fd];
+            const float f = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
+            accd += f * reinterpret_cast<const float*>(&s_acc[q * F + fd])[cd];
+            wt += f * s_s[q * F + fd];
+        }
     }
     const float res = wt > 0.f ? accd / wt : 0.f;
-    a.out[orow * kD + tid] = __float2bfloat16_rn(res);
-    if (a.lse != nullptr && tid == 0) a.lse[orow] = wt > 0.f ? (mx + log2f(wt)) * kLn2 : -INFINITY;
+    a.out[orow * kD + d_lo + tid] = __float2bfloat16_rn(res);
+    if (a.lse != nullptr && tid == 0 && blockIdx.z == 0)
+        a.lse[orow] = wt > 0.f ? (M + log2f(wt)) * kLn2 : -INFINITY;
+    if (threadIdx.x == 0) WMTP_TRACE_AT(51);
 }
 
 }  // namespace wmtp

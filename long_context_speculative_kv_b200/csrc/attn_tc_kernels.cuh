@@ -199,13 +199,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    pdl_launch_dependents();
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
     pdl_wait();
+    pdl_launch_dependents();   // after the wait, as attn_split_kernel (the LSE merge plans early)
 
     // ---- plan (as attn_split_kernel) -----------------------------------------------------
     if (warp == 0) {

@@ -277,6 +277,14 @@ int ctas_per_sm(Kern k) {
 }
 constexpr int kMaxCtasPerSm = 3;
 
+// LSE-merge grid: (units, rows per block, C head-dim chunks), with the smallest C whose one round
+// of loads (8 C x kMergeBatch partials) covers a unit's expected partials (~P / units + 1).
+dim3 merge_grid(const Shape& s, int P) {
+    const long long per_unit = (long long)P / (s.units > 0 ? s.units : 1) + 1;
+    const int C = per_unit <= 8 * kMergeBatch ? 1 : (per_unit <= 16 * kMergeBatch ? 2 : 4);
+    return dim3((unsigned)s.units, (unsigned)s.rows_blk, (unsigned)C);
+}
+
 template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
 int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                   const Shape& s, cudaStream_t st) {
@@ -288,7 +296,7 @@ int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& 
     const int grid = sm_count * MINB;
     rc = launch(kern, dim3(grid), dim3((NMT * NKG + 1) * 32), Lay::kAlloc, st, km, vm, a);
     if (rc != WMTP_OK) return rc;
-    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kMergeThreads), 0, st, a, grid);
+    return launch(lse_merge_kernel<SRC>, merge_grid(s, grid), dim3(kMergeThreads), 0, st, a, grid);
 }
 
 template <int SRC, int NK, int NV, int NSB, bool KV8 = false>
@@ -305,7 +313,7 @@ int launch_attn_tc_t(const CUtensorMap& km, const CUtensorMap& vm, const void* q
     const int grid = sm_count;
     rc = launch(kern, dim3(grid), dim3(tc_threads<KV8>()), Lay::kAlloc, st, km, vm, qm, a);
     if (rc != WMTP_OK) return rc;
-    return launch(lse_merge_kernel<SRC>, dim3(s.units, s.rows_blk), dim3(kMergeThreads), 0, st, a, grid);
+    return launch(lse_merge_kernel<SRC>, merge_grid(s, grid), dim3(kMergeThreads), 0, st, a, grid);
 }
 
 template <int SRC>

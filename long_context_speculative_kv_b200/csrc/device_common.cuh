@@ -143,8 +143,10 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
 // ---------------------------------------------------------------------------------------------
 // Programmatic dependent launch.  Every kernel of the library lets the next kernel on the stream
 // launch early (its CTAs then block in pdl_wait) and waits for its own predecessor to finish,
-// with memory visible, before it touches global memory.  Without the launch attribute both are
-// no-ops.
+// with memory visible, before it touches global memory that kernel may write.  The attention
+// kernels trigger only after their own wait, so the LSE merge that follows one may read the
+// request lengths (final by then, and not written by the attention kernel) before its wait.
+// Without the launch attribute both are no-ops.
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
