@@ -245,6 +245,26 @@ struct TileWalker {
     }
 };
 
+// The unit of flat tile t (b, h, rb, unit and L_tot only; no page-table read), so that the
+// consumers can start their first unit (its Q loads) while the first tile is still in flight.
+__device__ __forceinline__ void unit_of_tile(const AttnArgs& a, const int* plan_tiles,
+                                             const int* plan_len, long long t, TileMeta& m) {
+    const int units_b = a.Hkv * a.n_rb;
+    int b = 0;
+    long long b_start = 0, per_b = (long long)plan_tiles[0] * units_b;
+    while (t >= b_start + per_b) {
+        b_start += per_b;
+        ++b;
+        per_b = (long long)plan_tiles[b] * units_b;
+    }
+    const int unit_in_b = (int)((t - b_start) / plan_tiles[b]);
+    m.b = b;
+    m.h = unit_in_b / a.n_rb;
+    m.rb = unit_in_b - m.h * a.n_rb;
+    m.unit = (b * a.Hkv + m.h) * a.n_rb + m.rb;
+    m.L_tot = plan_len[b];
+}
+
 // ---------------------------------------------------------------------------------------------
 // Cluster window mode: one unit per cluster of CL_size CTAs (grid (CL_size, units)), CTA r of
 // the cluster takes the unit's tiles [floor(r nt / CL_size), floor((r + 1) nt / CL_size)).  The
@@ -449,9 +469,11 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) WMTP_TRACE_AT(0);
+    uint64_t pol = 0;                          // the producer's L2 policy for the KV stream
     if (warp == NWC && lane == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
+        pol = l2_evict_first_policy();
     }
     // the successor may launch once this kernel's predecessor is done (so it may read, before
     // its own wait, inputs this kernel does not write: the LSE merge reads the lengths early)
@@ -531,17 +553,19 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     if (warp == NWC) {
         // =========================== producer warp =========================================
         if (lane == 0 && t_begin < t_end) {
-            const uint64_t pol = l2_evict_first_policy();
+            if (threadIdx.x == 32 * NWC) WMTP_TRACE_AT(42);
             TileWalker<SRC> walk;
             if (!CL) walk.init(a, plan_tiles);
             uint32_t it = 0;
             for (long long t = t_begin; t < t_end; ++t, ++it) {
                 TileMeta m;
                 int ty = 0, tz = 0;
+                if (it == 0) WMTP_TRACE_AT(40);
                 if (CL)
                     s_walk.describe(a, (int)t, (int)t_begin, (int)t_end, m, ty, tz);
                 else
                     walk.describe(a, plan_tiles, plan_len, t, t_begin, t_end, m, ty, tz);
+                if (it == 0) WMTP_TRACE_AT(41);
                 const int stage = (int)(it % NSTAGE);
                 const uint32_t phase = (it / NSTAGE) & 1u;
                 if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u)) break;
@@ -693,12 +717,17 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             }
                 return true;
     };
-    if (CL && t_begin < t_end) {
-        // cluster mode: the unit is known from the plan, so its Q loads overlap the first tile's
+    if (t_begin < t_end) {
+        // the first unit is known from the plan, so its Q loads overlap the first tile's TMA
         TileMeta m0;
-        int ty0 = 0, tz0 = 0;
-        s_walk.describe(a, (int)t_begin, (int)t_begin, (int)t_end, m0, ty0, tz0);
+        if (CL) {
+            int ty0 = 0, tz0 = 0;
+            s_walk.describe(a, (int)t_begin, (int)t_begin, (int)t_end, m0, ty0, tz0);
+        } else {
+            unit_of_tile(a, plan_tiles, plan_len, t_begin, m0);
+        }
         if (!unit_start(m0)) alive = false;
+        if (warp == 0 && lane == 0) WMTP_TRACE_AT(12);
     }
     for (long long t = t_begin; t < t_end && alive; ++t, ++it) {
         const int stage = (int)(it % NSTAGE);
@@ -741,7 +770,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             }
         }
 
-        if ((m.flags & kFirst) && !(CL && it == 0)) {
+        if ((m.flags & kFirst) && it != 0) {
             if (!unit_start(m)) { alive = false; break; }
         }
 
@@ -1066,6 +1095,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         }
     }
     if (warp == 0 && lane == 0) WMTP_TRACE_AT(28);
+    if (warp == 0 && lane == 0) WMTP_TRACE_MAX(43);
     if (CL) {
         __syncwarp();
         cluster_merge_rows<NMT, NKG, NSTAGE, KV8, QS>(a, smem, s_walk, s_peff, warp, lane);

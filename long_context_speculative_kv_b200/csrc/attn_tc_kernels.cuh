@@ -199,6 +199,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    uint64_t pol = 0;                          // the producers' L2 policy for the KV stream
+    if ((warp == 0 || warp == 6) && lane == 0) pol = l2_evict_first_policy();
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
@@ -267,7 +269,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         // =========================== producers ===============================================
         if (lane == 0) {
             const bool is_k = (warp == 0);
-            const uint64_t pol = l2_evict_first_policy();
             TileWalker<SRC> walk;
             walk.init(a, plan_tiles);
             uint32_t uidx = 0, it = 0;

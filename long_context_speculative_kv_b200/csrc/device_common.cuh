@@ -55,7 +55,12 @@ __device__ unsigned long long g_trace[kTraceSlots];
         const int tt_ = (int)(t) - kTraceT0;                                        \
         if (tt_ >= 0 && tt_ < 32) WMTP_TRACE_AT(64 + 32 * (role) + tt_);             \
     } while (0)
+// the latest time any CTA passed this point (slot i)
+#define WMTP_TRACE_MAX(i) atomicMax(&g_trace[(i)], (unsigned long long)global_ns())
 #else
+#define WMTP_TRACE_MAX(i) \
+    do {                  \
+    } while (0)
 #define WMTP_TRACE_AT(i) \
     do {                 \
     } while (0)
