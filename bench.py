@@ -224,6 +224,22 @@ class Timing:
         torch.cuda.synchronize()
         return g, api.launch_count() - n0
 
+    def capture_e2e(self, step, arm, h_in, h_out):
+        """One end-to-end step captured as a CUDA graph: the H2D copies of the step's inputs from
+        the pinned host buffers, the step's C-ABI calls and the D2H copies of the accepted tokens
+        (memcpy nodes; each replay copies whatever the host buffers hold then)."""
+        import torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step.run_e2e(arm, h_in, h_out)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.run_e2e(arm, h_in, h_out)
+        torch.cuda.synchronize()
+        return g
+
     def timed_graph(self, step, g, K, e2e=None):
         import torch
         self.barrier()
@@ -509,11 +525,17 @@ def measure_headline(args, T, peaks, rank, world, local, device):
         torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers --------------------------------
+    step.pack_io()          # one H2D and one D2H copy per step
     h_in, h_out = step.host_inputs(), step.host_outputs()
     for _ in range(2):
         step.run_e2e("windowed", h_in, h_out)
     ms_e2e_eager, _, _ = T.timed(step, "windowed", args.steps, e2e=(h_in, h_out))
-    ms_e2e = T.timed_graph(step, g_w, args.steps, e2e=(h_in, h_out)) if use_graph else ms_e2e_eager
+    if use_graph:
+        g_e2e = T.capture_e2e(step, "windowed", h_in, h_out)
+        ms_e2e = T.timed_graph(step, g_e2e, args.steps)
+        del g_e2e
+    else:
+        ms_e2e = ms_e2e_eager
     e2e_value = per_replica_us_per_step(T.max_ranks(ms_e2e), args.steps)
     e2e_eager_value = per_replica_us_per_step(T.max_ranks(ms_e2e_eager), args.steps)
     if use_graph:
@@ -794,12 +816,13 @@ def measure_headline(args, T, peaks, rank, world, local, device):
         "gamma_sweep": sweep, "context_sweep": ctx_sweep, "decode_loop": loop_res, "fp8_kv": fp8_res,
         "kv_accounting": accounting,
         "roofline": roofline, "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_value, 3), "unit": "us/step",
+        "e2e": {"value": round(e2e_eager_value, 3), "unit": "us/step",
                 "h2d_bytes_per_step": DecodeStep.bytes_of(h_in), "d2h_bytes_per_step": DecodeStep.bytes_of(h_out),
-                "mode": "CUDA-graph replay of the step's C-ABI calls; pinned-host inputs copied in and "
-                        "accepted tokens copied out every step, inside the timed region",
-                "eager_value": round(e2e_eager_value, 3),
-                "eager_mode": "the same with every C-ABI call issued from the host each step"},
+                "mode": "every C-ABI call of the step issued from the host each step, with one copy of the "
+                        "step's inputs from pinned host memory before them and one copy of the accepted "
+                        "tokens to pinned host memory after them, all inside the timed region",
+                "graph_value": round(e2e_value, 3),
+                "graph_mode": "the same step (copies included) captured once as a CUDA graph and replayed"},
         "gpu_launches": launches, "gpu_launches_per_step": launches / args.steps,
         "gpu_launches_per_step_native": per_step_launches_n,
         "clocks": clk, "kernel_source": kernel_source_hash(),

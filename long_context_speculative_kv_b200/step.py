@@ -193,25 +193,56 @@ class DecodeStep:
         if log: log.mark(None)
 
     # ----------------------------------------------------------------------------- e2e
-    def host_inputs(self) -> Dict[str, torch.Tensor]:
-        """Pinned host copies of every per-step input (what a serving loop hands over)."""
+    _INPUTS = ("q_verify", "logits", "tokens", "q_ctx", "q_fwd", "k_ctx", "v_ctx", "k_fwd", "v_fwd")
+    _OUTPUTS = ("accepted", "n_accepted")
+
+    def pack_io(self):
+        """Re-homes the per-step inputs and the acceptance outputs into one contiguous device
+        buffer each (views at 256-byte offsets, contents kept), so that a step's host transfers
+        are one copy in and one copy out."""
         b = self.b
-        names = ["q_verify", "logits", "tokens", "q_ctx", "q_fwd", "k_ctx", "v_ctx", "k_fwd", "v_fwd"]
-        return {n: getattr(b, n).cpu().pin_memory() for n in names}
+
+        def pack(tensors):
+            offs, total = [], 0
+            for t in tensors:
+                offs.append(total)
+                total += (t.numel() * t.element_size() + 255) // 256 * 256
+            buf = torch.empty(total, dtype=torch.uint8, device=tensors[0].device)
+            views = []
+            for t, o in zip(tensors, offs):
+                v = buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                v.copy_(t)
+                views.append(v)
+            return buf, views
+
+        self._in_buf, views = pack([getattr(b, n) for n in self._INPUTS])
+        for n, v in zip(self._INPUTS, views):
+            setattr(b, n, v)
+        self._out_buf, views = pack([b.out[n] for n in self._OUTPUTS])
+        for n, v in zip(self._OUTPUTS, views):
+            b.out[n] = v
+
+    def host_inputs(self) -> Dict[str, torch.Tensor]:
+        """Pinned host copies of every per-step input (what a serving loop hands over): one
+        buffer with the device layout after pack_io, else one tensor per input."""
+        if getattr(self, "_in_buf", None) is not None:
+            return {"packed_inputs": self._in_buf.cpu().pin_memory()}
+        return {n: getattr(self.b, n).cpu().pin_memory() for n in self._INPUTS}
 
     def host_outputs(self) -> Dict[str, torch.Tensor]:
+        if getattr(self, "_out_buf", None) is not None:
+            return {"packed_outputs": torch.empty(self._out_buf.shape, dtype=torch.uint8).pin_memory()}
         b = self.b
-        return {n: torch.empty(b.out[n].shape, dtype=b.out[n].dtype).pin_memory()
-                for n in ("accepted", "n_accepted")}
+        return {n: torch.empty(b.out[n].shape, dtype=b.out[n].dtype).pin_memory() for n in self._OUTPUTS}
 
     def run_e2e(self, arm: str, h_in: Dict[str, torch.Tensor], h_out: Dict[str, torch.Tensor]):
         """H2D of the step's inputs, the step, D2H of the accepted tokens (all async)."""
         b = self.b
         for n, t in h_in.items():
-            getattr(b, n).copy_(t, non_blocking=True)
+            (self._in_buf if n == "packed_inputs" else getattr(b, n)).copy_(t, non_blocking=True)
         self.run(arm)
         for n, t in h_out.items():
-            t.copy_(b.out[n], non_blocking=True)
+            t.copy_(self._out_buf if n == "packed_outputs" else b.out[n], non_blocking=True)
 
     @staticmethod
     def bytes_of(ts: Dict[str, torch.Tensor]) -> int:
