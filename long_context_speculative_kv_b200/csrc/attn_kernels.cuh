@@ -245,6 +245,50 @@ struct TileWalker {
     }
 };
 
+// Before the PDL wait (paged source, one thread): this CTA's first n tiles, planned from the
+// lengths and page table as they read at that moment, are prefetched into L2, so that their DRAM
+// latency overlaps the predecessor's tail.  The predecessor may still be writing those inputs; a
+// stale read only warms the wrong lines (nothing is loaded into shared memory or used), and every
+// read stays inside the table and every prefetch inside a valid page.  Requests beyond 16 skip it.
+__device__ __forceinline__ void prefetch_first_tiles(const AttnArgs& a, const CUtensorMap* kmap,
+                                                     const CUtensorMap* vmap, bool kv8, int n) {
+    if (a.B > 16) return;
+    const int units_b = a.Hkv * a.n_rb;
+    long long T = 0;
+    for (int b = 0; b < a.B; ++b) {
+        const int L = a.kv_len[b];
+        T += (long long)((L > 0 ? L : 0) + kTileKeys - 1) / kTileKeys * units_b;
+    }
+    const int peff = plan_ctas(T, gridDim.x, a.min_tiles_per_cta);
+    const long long c = blockIdx.x;
+    if (c >= peff) return;
+    long long t = cta_begin(c, T, peff);
+    const long long t1 = cta_begin(c + 1, T, peff);
+    for (int k = 0; k < n && t < t1; ++k, ++t) {
+        long long b_start = 0;
+        int b = 0, nt = 0;
+        for (; b < a.B; ++b) {
+            const int L = a.kv_len[b];
+            nt = ((L > 0 ? L : 0) + kTileKeys - 1) / kTileKeys;
+            if (t < b_start + (long long)nt * units_b) break;
+            b_start += (long long)nt * units_b;
+        }
+        if (b >= a.B || nt == 0) return;
+        const int unit_in_b = (int)((t - b_start) / nt);
+        const int tile = (int)((t - b_start) - (long long)unit_in_b * nt);
+        if (tile >= a.max_pages) return;
+        const int page = a.page_table[(size_t)b * a.max_pages + tile];
+        if (page < 0 || page >= a.num_pages) return;
+        const int tz = page * a.Hkv + unit_in_b / a.n_rb;
+        tma_prefetch_3d(kmap, 0, 0, tz);
+        tma_prefetch_3d(vmap, 0, 0, tz);
+        if (!kv8) {
+            tma_prefetch_3d(kmap, 64, 0, tz);
+            tma_prefetch_3d(vmap, 64, 0, tz);
+        }
+    }
+}
+
 // The unit of flat tile t (b, h, rb, unit and L_tot only; no page-table read), so that the
 // consumers can start their first unit (its Q loads) while the first tile is still in flight.
 __device__ __forceinline__ void unit_of_tile(const AttnArgs& a, const int* plan_tiles,
@@ -474,6 +518,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
         pol = l2_evict_first_policy();
+        if (!CL && SRC == kSrcPaged) prefetch_first_tiles(a, &kmap, &vmap, KV8, NSTAGE);
     }
     // the successor may launch once this kernel's predecessor is done (so it may read, before
     // its own wait, inputs this kernel does not write: the LSE merge reads the lengths early)

@@ -205,6 +205,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
+        if (SRC == kSrcPaged) prefetch_first_tiles(a, &kmap, &vmap, KV8, 4);
     }
     pdl_wait();
     pdl_launch_dependents();   // after the wait, as attn_split_kernel (the LSE merge plans early)
