@@ -1245,26 +1245,40 @@ lse_merge_kernel(const AttnArgs a, int P_launch) {
         }
     }
     if (threadIdx.x == 0) WMTP_TRACE_AT(50);
+    // the threads of one partial lane (same qk) folded the same partials: one (max, sum) per
+    // lane, kept by its first thread; warp 0 turns them into weights once
     __shared__ float4 s_acc[kMergeThreads];
-    __shared__ float s_m[kMergeThreads], s_s[kMergeThreads];
+    __shared__ float s_m[32], s_s[32], s_f[32], s_wt;
+    __shared__ float s_M;
     s_acc[tid] = acc;
-    s_m[tid] = m_t;
-    s_s[tid] = s_t;
+    if (f4 == 0) {
+        s_m[qk] = m_t;
+        s_s[qk] = s_t;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        const float mq = tid < lanes ? s_m[tid] : -INFINITY;
+        float M = mq;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float f = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
+        float wt = tid < lanes ? f * s_s[tid] : 0.f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) wt += __shfl_xor_sync(0xffffffffu, wt, off);
+        s_f[tid] = f;
+        if (tid == 0) {
+            s_M = M;
+            s_wt = wt;
+        }
+    }
     __syncthreads();
     if (tid >= dims) return;
     // thread d combines head dim d_lo + d over the partial lanes
     const int fd = tid >> 2, cd = tid & 3;
-    float M = -INFINITY;
-    for (int q = 0; q < lanes; ++q) M = fmaxf(M, s_m[q * F + fd]);
-    float accd = 0.f, wt = 0.f;
-    if (M != -INFINITY) {
-        for (int q = 0; q < lanes; ++q) {
-            const float mq = s_m[q * F + fd];
-            const float f = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
-            accd += f * reinterpret_cast<const float*>(&s_acc[q * F + fd])[cd];
-            wt += f * s_s[q * F + fd];
-        }
-    }
+    float accd = 0.f;
+    for (int q = 0; q < lanes; ++q)
+        accd += s_f[q] * reinterpret_cast<const float*>(&s_acc[q * F + fd])[cd];
+    const float wt = s_wt, M = s_M;
     const float res = wt > 0.f ? accd / wt : 0.f;
     a.out[orow * kD + d_lo + tid] = __float2bfloat16_rn(res);
     if (a.lse != nullptr && tid == 0 && blockIdx.z == 0)
