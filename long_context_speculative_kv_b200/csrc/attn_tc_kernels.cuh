@@ -692,17 +692,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
             for (int j = 0; j < 16; ++j) {
                 const float p0 = fast_exp2(fmaf(x[2 * j], rs, -m_sub));
                 const float p1 = fast_exp2(fmaf(x[2 * j + 1], rs, -m_sub));
-                if (KV8) {
-                    // fp16 weights for the fp16 V; the row sum over the fp32 weights (fp16 keeps 11
-                    // bits, so the two sums differ by far less than the tolerance, and the
-                    // conversions back to fp32 would compete with the V widening for the
-                    // conversion pipe)
-                    pk[j] = pack_f16x2(p0, p1);
-                    ls[j & 3] += p0 + p1;
-                } else {
-                    pk[j] = pack_bf16x2(p0, p1);
-                    ls[j & 3] += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
-                }
+                // fp16 (fp8 KV) or bf16 weights for PV; the row sum over the fp32 weights (the
+                // rounded weights would cost two unpacks a pair; the sums differ by at most 2^-9
+                // of a weight, within the tolerance)
+                pk[j] = KV8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+                ls[j & 3] += p0 + p1;
             }
             l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             if (lane == 0 && warp == gwarp0) WMTP_TRACE_TILE(10, it);

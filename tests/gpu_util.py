@@ -10,9 +10,9 @@ bf16 next to the bf16 values, and the output itself.  So, with e = |gpu - ref|:
     rounding, a quarter ulp on average, already exceeds 2e-3 at |ref| > 1, so a plain mean could
     not hold for outputs of that size whatever the kernel computed before rounding).
 For unit-scale outputs (|ref| < 1) u(ref) <= 2^-8, so the bounds are within 2e-3 of the plain
-ones.  LSE (fp32): |gpu - ref| <= 4e-3 + 1e-5 |ref| (the row sums are sums of the bf16-rounded
-weights the PV product uses, so ln of a sum carries up to 2^-8 of their rounding), equal
-infinities allowed.
+ones.  LSE (fp32): |gpu - ref| <= 4e-3 + 1e-5 |ref| (the tcgen05 kernel's row sums are sums of
+the bf16-rounded weights the PV product uses, so ln of a sum carries up to 2^-8 of their
+rounding), equal infinities allowed.
 """
 import numpy as np
 import torch
