@@ -91,6 +91,21 @@ def test_verify_chain_matches_oracle(L, n_q, Hq, Hkv):
     assert_lse_close(lse, ref_lse)
 
 
+@pytest.mark.parametrize("n_q", [4, 8])
+def test_verify_many_ragged_requests(n_q):
+    """Twenty requests of ragged lengths (more than the kernels' early L2 prefetch plans for):
+    32-row units on the mma.sync kernel, 64-row units on the tcgen05 kernel, units split over
+    several CTAs and units finished inside one."""
+    sc = 128 ** -0.5
+    rng = np.random.default_rng(11)
+    lens = [int(x) + n_q for x in rng.integers(1, 3000, size=20)]
+    c = paged_case(3, lens, 32, 4, n_q)
+    out, lse = run_paged(c, "verify", sc)
+    ref, ref_lse = oracle.attention(c["q"], c["k"], c["v"], c["lens"], oracle.MODE_CAUSAL, sc)
+    assert_attn_close(out, ref, "verify, 20 ragged requests")
+    assert_lse_close(lse, ref_lse)
+
+
 def test_verify_tree_matches_oracle():
     sc = 128 ** -0.5
     lens_committed = [3000, 1234, 777]
