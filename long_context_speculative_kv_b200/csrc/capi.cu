@@ -265,10 +265,14 @@ Kern select_kernel(const Shape& s, bool kv8) {
 #define WMTP_SPLIT32_ONE_CTA 0
 #endif
 
-// CTAs per SM of each kernel (the grid is sm_count times this).
-int ctas_per_sm(Kern k) {
+// CTAs per SM of each kernel (the grid is sm_count times this).  Units of at most 16 rows read
+// from the ring run two CTAs of two stages per SM: a large window is mostly L2-resident, and the
+// 8-row consumer (~0.7 us a tile) rather than HBM then sets the pace, so two pipelines per SM
+// help (64 MiB window call 19.6 -> 15.4 us); from the paged cache one CTA of four stages per SM
+// already streams at the HBM rate.
+int ctas_per_sm(Kern k, bool ring = false) {
     switch (k) {
-        case Kern::kSplit16: return 1;
+        case Kern::kSplit16: return ring ? 2 : 1;
         case Kern::kSplit32: return WMTP_SPLIT32_ONE_CTA ? 1 : 2;
         case Kern::kSplit16Fp8: return 3;
         case Kern::kTc: case Kern::kTcFp8: return 1;
@@ -320,7 +324,9 @@ template <int SRC>
 int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                 const Shape& s, cudaStream_t st, bool kv8 = false) {
     switch (select_kernel(s, kv8)) {
-        case Kern::kSplit16: return launch_attn_t<SRC, 1, 4, 4, 1>(km, vm, a, sm_count, s, st);
+        case Kern::kSplit16:
+            if (SRC == kSrcRing) return launch_attn_t<SRC, 1, 4, 2, 2>(km, vm, a, sm_count, s, st);
+            return launch_attn_t<SRC, 1, 4, 4, 1>(km, vm, a, sm_count, s, st);
         case Kern::kSplit32:
 #if WMTP_SPLIT32_ONE_CTA
             return launch_attn_t<SRC, 2, 2, 4, 1>(km, vm, a, sm_count, s, st);
@@ -439,7 +445,7 @@ int launch_window_cluster(const CUtensorMap& km, const CUtensorMap& vm, const At
 // Common front half of the three attention calls.
 int prepare(const Shape& s, const void* q, const void* out, const float* lse, void* ws,
             size_t ws_bytes, float sm_scale, DeviceInfo* dev, AttnArgs* a, bool kv8 = false,
-            float k_scale = 1.f, float v_scale = 1.f) {
+            float k_scale = 1.f, float v_scale = 1.f, bool ring = false) {
     if (q == nullptr || out == nullptr || ws == nullptr) return WMTP_ERR_ARG;
     if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return WMTP_ERR_ARG;
     if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
@@ -449,7 +455,7 @@ int prepare(const Shape& s, const void* q, const void* out, const float* lse, vo
         return WMTP_ERR_ALIGN;
     int rc = device_info(dev);
     if (rc != WMTP_OK) return rc;
-    const int grid = dev->sm_count * ctas_per_sm(select_kernel(s, kv8));
+    const int grid = dev->sm_count * ctas_per_sm(select_kernel(s, kv8), ring);
     if (grid > kMaxParts) return WMTP_ERR_SHAPE;           // the merge's per-row weight table
     const long long slots = (long long)grid + s.units;
     if (ws_bytes < ws_total_bytes(slots, s.rows_blk)) return WMTP_ERR_WORKSPACE;
@@ -625,6 +631,10 @@ int ring_append_call(void* ring_k, void* ring_v, int64_t* ring_len, const void* 
 // (n_new > 0: positions [ring_len[b], ring_len[b] + n_new) get the rows of k_new / v_new and
 // ring_len advances, as ring_kv_append would).  stream_k: the stream-K kernel with workspace
 // partials and the LSE merge kernel instead of the cluster kernel (the no-alloc entry point).
+// Windowed calls of few units whose key sets hold at least this many tiles per SM in all (units x
+// the longest key set's tiles / SMs) take the stream-K path.
+constexpr int kWindowStreamKTilesPerSm = 7;
+
 int window_call(const wmtp_bf16* q, void* ring_k, void* ring_v, int64_t* ring_len,
                 const void* k_new, const void* v_new, int n_new,
                 int B, int n_q, int Hq, int Hkv, int D, int n_sink, int window, int capacity,
@@ -643,13 +653,22 @@ int window_call(const wmtp_bf16* q, void* ring_k, void* ring_v, int64_t* ring_le
         if (!aligned(k_new, 16) || !aligned(v_new, 16)) return WMTP_ERR_ALIGN;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // the fused append covers new rows that all fall in the call's key set (n_new <= window);
-    // otherwise the append runs as its own kernel first
-    const bool fused = n_new > 0 && n_new <= window && !stream_k && s.units <= 65535;
     DeviceInfo dev;
     AttnArgs a;
-    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a, kv8, k_scale, v_scale);
+    rc = prepare(s, q, out, lse, ws, ws_bytes, sm_scale, &dev, &a, kv8, k_scale, v_scale, true);
     if (rc != WMTP_OK) return rc;
+    // tiles of the longest key set: the sink's, the window's, one more where the window wraps
+    const int max_tiles = (n_sink + kTileKeys - 1) / kTileKeys + (window + kTileKeys - 1) / kTileKeys + 1;
+    // the cluster kernel (one launch) unless its clusters of at most 16 CTAs leave SMs idle (few
+    // units) while the call holds many tiles (a long window): then the stream-K kernel over every
+    // SM plus the LSE merge (64 MiB NoPE call, 8 units: 20.1 -> 15.5 us; 8 requests x 8 MiB,
+    // 32 units: the cluster kernel, 14.3 vs 17.8 us; 8 MiB, 4 units: cluster, 9.7 vs 12.1 us)
+    const bool use_sk = stream_k || s.units > 65535 ||
+                        ((long long)s.units * WMTP_CL_MAX < dev.sm_count &&
+                         (long long)s.units * max_tiles >= (long long)kWindowStreamKTilesPerSm * dev.sm_count);
+    // the fused append covers new rows that all fall in the call's key set (n_new <= window);
+    // otherwise the append runs as its own kernel first
+    const bool fused = n_new > 0 && n_new <= window && !use_sk;
     if (n_new > 0 && !fused) {
         rc = kv8 ? ring_append_call<8>(ring_k, ring_v, ring_len, k_new, v_new, B, n_new, Hkv, D, n_sink,
                                        capacity, stream)
@@ -672,10 +691,7 @@ int window_call(const wmtp_bf16* q, void* ring_k, void* ring_v, int64_t* ring_le
     CUtensorMap km, vm;
     if ((rc = encode_rows_map(&km, ring_k, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
     if ((rc = encode_rows_map(&vm, ring_v, capacity, (long long)B * Hkv, kv8)) != WMTP_OK) return rc;
-    if (stream_k || s.units > 65535)
-        return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, st, kv8);
-    // tiles of the longest key set: the sink's, the window's, one more where the window wraps
-    const int max_tiles = (n_sink + kTileKeys - 1) / kTileKeys + (window + kTileKeys - 1) / kTileKeys + 1;
+    if (use_sk) return launch_attn<kSrcRing>(km, vm, a, dev.sm_count, s, st, kv8);
     return launch_window_cluster(km, vm, a, s, max_tiles, st, kv8);
 }
 
