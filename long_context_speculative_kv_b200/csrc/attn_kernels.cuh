@@ -359,22 +359,27 @@ __device__ __forceinline__ unsigned long long step_visibility(const AttnArgs& a,
 // Shared-memory layout (dynamic; stage buffers 1024-byte aligned for the 128-byte swizzle).
 // QS (fp8 KV only): the unit's Q rows are kept in shared memory as fp16, in a space the unit-end
 // key-group merge reuses one m-tile at a time.
-template <int NMT, int NKG, int NSTAGE, bool KV8 = false, bool QS = false>
+// MS: the key-group merge at a unit's end goes through the stage of the unit's last tile (held
+// until the merge is done) instead of a space of its own, which leaves room for a third stage in
+// two CTAs per SM.
+template <int NMT, int NKG, int NSTAGE, bool KV8 = false, bool QS = false, bool MS = false>
 struct SmemLayout {
     static constexpr int kStagesBytes = NSTAGE * (KV8 ? kStageBytes8 : kStageBytes);
     static constexpr int kMergeStride = kD + 4;                      // floats per merge row
     static constexpr int kMergeMT = QS ? 1 : NMT;                    // m-tiles merged at once
     static constexpr int kMergeFloats = (NKG - 1) * kMergeMT * 16 * kMergeStride;
     static constexpr int kMergeMLFloats = (NKG - 1) * kMergeMT * 16 * 2;
+    static_assert(!MS || (!QS && (kMergeFloats + kMergeMLFloats) * 4 <= (KV8 ? kStageBytes8 : kStageBytes)),
+                  "the merge rows fit one stage");
     // fp16 Q row: 128 dims + 32 bytes of padding, so the 8-byte fragment reads of four rows in a
     // half-warp start 8 banks apart
     static constexpr int kQStride = 2 * kD + 32;
     static constexpr int kQBytes = QS ? NMT * 16 * kQStride : 0;
     static constexpr int kMergeOff = kStagesBytes;
     static constexpr int kQOff = kMergeOff;                          // QS: aliases the merge rows
-    static constexpr int kMergeBytes = (kQBytes > kMergeFloats * 4) ? kQBytes : kMergeFloats * 4;
+    static constexpr int kMergeBytes = MS ? kQBytes : ((kQBytes > kMergeFloats * 4) ? kQBytes : kMergeFloats * 4);
     static constexpr int kMergeMLOff = kMergeOff + kMergeBytes;
-    static constexpr int kBarOff = kMergeMLOff + kMergeMLFloats * 4;
+    static constexpr int kBarOff = kMergeMLOff + (MS ? 0 : kMergeMLFloats * 4);
     static constexpr int kMetaOff = kBarOff + (2 * NSTAGE + 1) * 8;
     static constexpr int kPlanOff = kMetaOff + NSTAGE * (int)sizeof(TileMeta);
     static constexpr int kPlanBytes = 2 * kMaxBatch * 4;            // tiles per request, length
@@ -481,11 +486,12 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* s
 // new row's key slot copy it from k_new / v_new into the tile (after the TMA landed) and into
 // the ring, and the last CTA to have read ring_len advances it.
 template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false,
-          bool CL = false>
+          bool CL = false, bool MS = false>
 __global__ void __launch_bounds__((NMT * NKG + 1) * 32, MINB)
 attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                   const AttnArgs a) {
-    using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
+    static_assert(!(MS && CL), "the cluster kernel keeps its merge space");
+    using L = SmemLayout<NMT, NKG, NSTAGE, KV8, QS, MS>;
     static_assert(!QS || KV8, "shared-memory Q is an fp8-KV layout");
     static_assert(!CL || SRC == kSrcRing, "the cluster kernel reads the ring");
     constexpr int kStage = KV8 ? kStageBytes8 : kStageBytes;
@@ -994,7 +1000,9 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         // write into it
         if (CL && patched) fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[stage]);
+        // MS: a unit's last stage is released after the key-group merge that goes through it
+        const bool hold_stage = MS && NKG > 1 && (m.flags & kLast);
+        if (lane == 0 && !hold_stage) mbar_arrive(&empty_bar[stage]);
         if (warp == 0 && lane == 0) WMTP_TRACE_TILE(2, it);
 
         if (m.flags & kLast) {
@@ -1052,9 +1060,13 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
                 if (!alive) break;
             } else if (NKG > 1) {
+                float* const mrg_o = MS ? reinterpret_cast<float*>(smem + (size_t)stage * kStage) : merge_o;
+                float* const mrg_ml = MS ? mrg_o + L::kMergeFloats : merge_ml;
+                // MS: every warp is past its reads of the stage's K and V before it is overwritten
+                if (MS && !consumers_sync()) { alive = false; break; }
                 if (kg > 0) {
-                    float* mo = merge_o + ((size_t)((kg - 1) * NMT + mt) * 16) * L::kMergeStride;
-                    float* ml = merge_ml + ((size_t)((kg - 1) * NMT + mt) * 16) * 2;
+                    float* mo = mrg_o + ((size_t)((kg - 1) * NMT + mt) * 16) * L::kMergeStride;
+                    float* ml = mrg_ml + ((size_t)((kg - 1) * NMT + mt) * 16) * 2;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
                         const int row = gid + 8 * r;
@@ -1069,8 +1081,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 if (kg == 0) {
 #pragma unroll 1
                     for (int g2 = 1; g2 < NKG; ++g2) {
-                        const float* mo = merge_o + ((size_t)((g2 - 1) * NMT + mt) * 16) * L::kMergeStride;
-                        const float* ml = merge_ml + ((size_t)((g2 - 1) * NMT + mt) * 16) * 2;
+                        const float* mo = mrg_o + ((size_t)((g2 - 1) * NMT + mt) * 16) * L::kMergeStride;
+                        const float* ml = mrg_ml + ((size_t)((g2 - 1) * NMT + mt) * 16) * 2;
 #pragma unroll
                         for (int r = 0; r < 2; ++r) {
                             const int row = gid + 8 * r;
@@ -1091,6 +1103,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     }
                 }
                 if (!consumers_sync()) { alive = false; break; }
+                // every warp has read the merge rows: the stage goes back to the producer
+                if (MS && lane == 0) mbar_arrive(&empty_bar[stage]);
             }
             if (CL && NKG == 1) {
                 // every consumer warp is past its last reads of the stage space the partial takes

@@ -265,6 +265,14 @@ Kern select_kernel(const Shape& s, bool kv8) {
 #define WMTP_SPLIT32_ONE_CTA 0
 #endif
 
+// Stages of the two-CTA layout of units of 17-32 rows (build-time for sweeps).  Its key groups
+// merge through the held stage of a unit's last tile, which leaves room for three 32 KiB stages in
+// two CTAs per SM (1M-key verify at 32 rows 313 -> 307 us; the ring layout of <= 16 rows gained
+// nothing from a third stage: 15.9 vs 15.9 us for the 64 MiB window call).
+#ifndef WMTP_SPLIT32_NSTAGE
+#define WMTP_SPLIT32_NSTAGE 3
+#endif
+
 // CTAs per SM of each kernel (the grid is sm_count times this).  Units of at most 16 rows read
 // from the ring run two CTAs of two stages per SM: a large window is mostly L2-resident, and the
 // 8-row consumer (~0.7 us a tile) rather than HBM then sets the pace, so two pipelines per SM
@@ -289,11 +297,12 @@ dim3 merge_grid(const Shape& s, int P) {
     return dim3((unsigned)s.units, (unsigned)s.rows_blk, (unsigned)C);
 }
 
-template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false>
+template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false,
+          bool MS = false>
 int launch_attn_t(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a, int sm_count,
                   const Shape& s, cudaStream_t st) {
-    using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8, QS>;
-    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB, KV8, QS>;
+    using Lay = SmemLayout<NMT, NKG, NSTAGE, KV8, QS, MS>;
+    auto kern = attn_split_kernel<SRC, NMT, NKG, NSTAGE, MINB, KV8, QS, false, MS>;
     static bool attr_set[kMaxDevices] = {};
     int rc = set_smem_once(kern, Lay::kAlloc, attr_set);
     if (rc != WMTP_OK) return rc;
@@ -331,7 +340,7 @@ int launch_attn(const CUtensorMap& km, const CUtensorMap& vm, const AttnArgs& a,
 #if WMTP_SPLIT32_ONE_CTA
             return launch_attn_t<SRC, 2, 2, 4, 1>(km, vm, a, sm_count, s, st);
 #else
-            return launch_attn_t<SRC, 2, 2, 2, 2>(km, vm, a, sm_count, s, st);
+            return launch_attn_t<SRC, 2, 2, WMTP_SPLIT32_NSTAGE, 2, false, false, true>(km, vm, a, sm_count, s, st);
 #endif
         case Kern::kSplit64: return launch_attn_t<SRC, 4, 1, 2, 2>(km, vm, a, sm_count, s, st);
         case Kern::kTc: return launch_attn_tc_t<SRC, 3, 3, 2>(km, vm, a.q, a, sm_count, s, st);
