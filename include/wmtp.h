@@ -286,7 +286,7 @@ WMTP_API int verify_attn_fp8(const wmtp_bf16* q, const uint8_t* k_pool, const ui
  *   Limit: the shape must fit the scratch: (CTAs the call launches, one or two per SM, plus
  *   B * Hkv * ceil(n_q * Hq / Hkv / 64)) partial slots of rows * 516 bytes each, rows =
  *   min(64, n_q * Hq / Hkv).  On a 148-SM B200 a one-query call with 8 query heads per kv head
- *   fits B * Hkv <= 1884, a 4-query call (32 rows) B * Hkv <= 212.  Larger shapes return
+ *   fits B * Hkv <= 1736, a 4-query call (32 rows) B * Hkv <= 212.  Larger shapes return
  *   WMTP_ERR_SCRATCH_LIMIT and launch nothing.
  *   The first call on each device looks up the scratch array's device address (with that device
  *   current); make that first call before any stream capture.
