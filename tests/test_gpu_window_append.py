@@ -55,6 +55,10 @@ def _append(kv8, *args):
     ([1, 2], 8, 2, 4, 252, 256, 6, 1, False),          # first rows land in the sink slots
     ([3000], 16, 2, 4, 1020, 1024, 4, 1, True),        # fp8 (E4M3) ring
     ([700, 1500], 32, 4, 4, 252, 260, 3, 4, True),     # fp8 context pass
+    # one unit with a window of 1041 tiles: the call takes the stream-K path (append kernel, then
+    # attention and LSE merge over every SM) instead of the cluster kernel
+    ([70000], 8, 1, 4, 66556, 66560, 3, 1, False),
+    ([70000], 8, 1, 4, 66556, 66560, 2, 1, True),
 ])
 def test_fused_forward_sequence(lens, Hq, Hkv, s, W, C, steps, n_new, kv8):
     sc = 128 ** -0.5
