@@ -57,7 +57,7 @@ def _both(q, ring_k, ring_v, rlen, Hkv, s, W, C, sc):
                                                out.data_ptr(), lse.data_ptr(), None)
         else:
             n = lib.wmtp_workspace_bytes(B, n_q, Hq, Hkv, D)
-            ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+            ws = torch.zeros(n, dtype=torch.uint8, device="cuda")   # control block zero
             rc = lib.draft_attn_window(q.data_ptr(), ring_k.data_ptr(), ring_v.data_ptr(),
                                        rlen.data_ptr(), B, n_q, Hq, Hkv, D, s, W, C, sc,
                                        out.data_ptr(), lse.data_ptr(), ws.data_ptr(), n, None)
