@@ -485,6 +485,19 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* s
 // a.n_new > 0 the call also appends the request's new draft rows: the consumer warps that own a
 // new row's key slot copy it from k_new / v_new into the tile (after the TMA landed) and into
 // the ring, and the last CTA to have read ring_len advances it.
+// Fused append: every CTA counts in once it has read ring_len; the last one to count in advances
+// ring_len by n_new for every request and clears the ticket for the next call.
+__device__ __forceinline__ void fused_append_ticket(const AttnArgs& a) {
+    __threadfence();
+    const unsigned int total = gridDim.x * gridDim.y;
+    if (atomicAdd(a.ticket, 1u) == total - 1u) {
+        __threadfence();
+        for (int b = 0; b < a.B; ++b) a.ring_len_w[b] = a.ring_len_w[b] + a.n_new;
+        *a.ticket = 0u;
+        __threadfence();
+    }
+}
+
 template <int SRC, int NMT, int NKG, int NSTAGE, int MINB, bool KV8 = false, bool QS = false,
           bool CL = false, bool MS = false>
 __global__ void __launch_bounds__((NMT * NKG + 1) * 32, MINB)
@@ -555,17 +568,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             s_range[0] = c * nt / cs;
             s_range[1] = (c + 1) * nt / cs;
             s_peff = nt;
-            if (a.n_new > 0) {
-                // every CTA has read its length: the last one to count in advances ring_len
-                __threadfence();
-                const unsigned int total = gridDim.x * gridDim.y;
-                if (atomicAdd(a.ticket, 1u) == total - 1u) {
-                    __threadfence();
-                    for (int b = 0; b < a.B; ++b) a.ring_len_w[b] = a.ring_len_w[b] + a.n_new;
-                    *a.ticket = 0u;
-                    __threadfence();
-                }
-            }
+            // a CTA with tiles counts in after its first TMA is issued (off the critical path)
+            if (a.n_new > 0 && s_range[0] >= s_range[1]) fused_append_ticket(a);
             for (int s = 0; s < NSTAGE; ++s) {
                 mbar_init(&full_bar[s], 1);
                 mbar_init(&empty_bar[s], NWC);
@@ -636,6 +640,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     mbar_arrive(&full_bar[stage]);
                 }
                 WMTP_TRACE_TILE(0, it);
+                if (CL && it == 0 && a.n_new > 0) fused_append_ticket(a);
             }
             // Drain: wait (bounded) until the consumers released every stage, so no TMA copy is
             // in flight into this CTA's shared memory when it exits.

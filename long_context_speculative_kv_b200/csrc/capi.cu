@@ -390,10 +390,10 @@ int cluster_capacity(K kern, int smem, int threads, int cs, int (&cache)[kMaxDev
 }
 
 // Build-time options for measurement sweeps: the largest cluster size, and the stage count /
-// CTAs per SM of the layout for units of at most 16 rows.  Two stages and two CTAs per SM
-// (94 KB of shared memory each) rather than the stream-K kernel's four stages and one CTA: the
-// smaller CTAs let eight 16-CTA clusters be resident at once (the NoPE workload's 8 units; at
-// 160 KB per CTA only clusters of 8 fit), 64 MiB window call 27.7 -> 20.2 us.
+// CTAs per SM of the cluster layout for units of at most 16 rows.  Two stages and two CTAs per SM
+// (94 KB of shared memory each) rather than four stages and one CTA: the smaller CTAs let eight
+// 16-CTA clusters be resident at once (at 160 KB per CTA only clusters of 8 fit; 8 units of a
+// 64 MiB window: 27.7 -> 20.2 us, a call that now takes the stream-K path, 15.5 us).
 #ifndef WMTP_CL_MAX
 #define WMTP_CL_MAX 16
 #endif
