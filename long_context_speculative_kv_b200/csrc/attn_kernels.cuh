@@ -35,6 +35,7 @@ constexpr int kStageBytes = 2 * kTileBytes;         // K + V: 32 KiB
 constexpr int kTileBytes8 = kTileKeys * kD;         // fp8 K or V tile: one 128x64 byte box, 8 KiB
 constexpr int kStageBytes8 = 2 * kTileBytes8;       // fp8 K + V: 16 KiB
 constexpr int kMaxBatch = 256;
+constexpr int kClusterMax = 16;                   // largest window cluster (non-portable size)
 constexpr float kLn2 = 0.693147180559945309f;
 
 enum SourceKind : int { kSrcPaged = 0, kSrcRing = 1 };
@@ -424,30 +425,31 @@ __device__ __forceinline__ void cluster_merge_rows(const AttnArgs& a, uint8_t* s
     const uint32_t part = smem_addr(smem + L::kPartOff);
     const uint32_t plse = smem_addr(smem + L::kPartLseOff);
     const bool has = lane < cs && (long long)(lane + 1) * nt / cs > (long long)lane * nt / cs;
+    const uint32_t has_mask = __ballot_sync(0xffffffffu, has);     // ranks holding a partial
     for (int rr = me + warp * cs; rr < rows_u; rr += kWarps * cs) {
+        // one round of remote loads: rank `lane`'s LSE and this lane's four head dims of every
+        // rank's partial are all in flight at once (a dependent round per step would cost one
+        // distributed-shared-memory round trip each)
         float x = -INFINITY;
         if (has) x = ld_dsmem_f32(map_shared_rank(plse + 4u * rr, lane));
+        const uint32_t po = part + 4u * (uint32_t)(rr * kD + 4 * lane);
+        float4 v[kClusterMax];
+#pragma unroll
+        for (int k = 0; k < kClusterMax; ++k)
+            v[k] = ((has_mask >> k) & 1u) ? ld_dsmem_v4(map_shared_rank(po, (uint32_t)k))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
         float mx = x;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         const float w = (has && mx != -INFINITY) ? exp2f(x - mx) : 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float wsum = 0.f;
-        const uint32_t po = part + 4u * (uint32_t)(rr * kD + 4 * lane);
-        // eight ranks' loads in flight at a time (a load waited on before the next is issued
-        // would cost one distributed-shared-memory round trip per rank)
-        for (int k0 = 0; k0 < cs; k0 += 8) {
-            float4 v[8];
-            float wv[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                wv[j] = (k0 + j < cs) ? __shfl_sync(0xffffffffu, w, k0 + j) : 0.f;
-                v[j] = wv[j] > 0.f ? ld_dsmem_v4(map_shared_rank(po, (uint32_t)(k0 + j))) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                acc.x += wv[j] * v[j].x; acc.y += wv[j] * v[j].y; acc.z += wv[j] * v[j].z; acc.w += wv[j] * v[j].w;
-                wsum += wv[j];
+        for (int k = 0; k < kClusterMax; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, w, k);
+            if (wk > 0.f) {
+                acc.x += wk * v[k].x; acc.y += wk * v[k].y; acc.z += wk * v[k].z; acc.w += wk * v[k].w;
+                wsum += wk;
             }
         }
         const int R = wk.rb * kRowsPerBlock + rr;

@@ -397,6 +397,7 @@ int cluster_capacity(K kern, int smem, int threads, int cs, int (&cache)[kMaxDev
 #ifndef WMTP_CL_MAX
 #define WMTP_CL_MAX 16
 #endif
+static_assert(WMTP_CL_MAX <= kClusterMax, "the cluster merge handles at most kClusterMax ranks");
 #ifndef WMTP_CL16_NSTAGE
 #define WMTP_CL16_NSTAGE 2
 #endif
