@@ -878,6 +878,29 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         mma_f16_16816(s[2 * np + 1], A1, b[6], b[7]);
                     }
                 }
+            } else if constexpr (SRC == kSrcRing && NT <= 2) {
+                // ring source (the windowed draft, whose few tiles per CTA make the consumer's
+                // latency the pace), 16 keys per warp: odd k-steps accumulate into a second
+                // set, so the dependent MMA chains are four long instead of eight
+                float s2[NT][4];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) s2[n][0] = s2[n][1] = s2[n][2] = s2[n][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        uint32_t b0a, b1a, b0b, b1b;
+                        ldsm_x4(tile_chunk_addr(kbase, key0 + np * 16 + k_row_l, ks * 2 + k_chk_l),
+                                b0a, b1a, b0b, b1b);
+                        float (*acc)[4] = (ks & 1) ? s2 : s;
+                        mma_bf16_16816(acc[2 * np], qa[ks], b0a, b1a);
+                        mma_bf16_16816(acc[2 * np + 1], qa[ks], b0b, b1b);
+                    }
+                }
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
             } else {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
@@ -1076,6 +1099,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     float* ml = mrg_ml + ((size_t)((kg - 1) * NMT + mt) * 16) * 2;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
+                        if (CL && !row_ok[r]) continue;     // (cluster mode: rows past the unit's)
                         const int row = gid + 8 * r;
 #pragma unroll
                         for (int n = 0; n < 16; ++n)
@@ -1092,6 +1116,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         const float* ml = mrg_ml + ((size_t)((g2 - 1) * NMT + mt) * 16) * 2;
 #pragma unroll
                         for (int r = 0; r < 2; ++r) {
+                            if (CL && !row_ok[r]) continue;
                             const int row = gid + 8 * r;
                             const float m2 = ml[row * 2], l2 = ml[row * 2 + 1];
                             const float mn = fmaxf(m_r[r], m2);
@@ -1109,7 +1134,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         }
                     }
                 }
-                if (!consumers_sync()) { alive = false; break; }
+                // the merge space is free again for the CTA's next unit (a cluster CTA has one)
+                if ((!CL || MS) && !consumers_sync()) { alive = false; break; }
                 // every warp has read the merge rows: the stage goes back to the producer
                 if (MS && lane == 0) mbar_arrive(&empty_bar[stage]);
             }
