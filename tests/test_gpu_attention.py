@@ -224,6 +224,23 @@ def test_draft_window_matches_oracle(lens, Hq, Hkv, n_q, s, W, C):
     assert_lse_close(lse, ref_lse)
 
 
+@pytest.mark.parametrize("W", [124, 316, 636, 1276, 2556])
+@pytest.mark.parametrize("n_q", [1, 4])
+def test_window_every_cluster_size(W, n_q):
+    """Windows of 2, 5, 10, 20 and 40 tiles: the cluster window kernel runs with clusters of 1, 2,
+    4, 8 and 16 CTAs per unit (the largest size that leaves each CTA at least two tiles), each
+    merging its partials through distributed shared memory; wrapped rings, ragged last tiles."""
+    sc = 128 ** -0.5
+    s = 4
+    lens = [3 * (s + W) + 37, 2 * (s + W) + 5]
+    c = ring_case(11 + W, lens, 32, 4, n_q, s, W, s + W)
+    out, lse = run_window(c, sc)
+    ref, ref_lse = oracle.attention(c["q"], c["k"], c["v"], c["lens"], oracle.MODE_WINDOW, sc,
+                                    n_sink=s, window=W)
+    assert_attn_close(out, ref, "draft_attn_window")
+    assert_lse_close(lse, ref_lse)
+
+
 def test_window_covering_context_equals_full():
     """s + W >= L: the windowed call equals the full call (both vs the oracle, and each other)."""
     sc = 128 ** -0.5
