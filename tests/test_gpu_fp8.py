@@ -150,6 +150,37 @@ def test_ring_fp8_append_and_window_attention(L, n_q, s, W, C):
     assert_lse_close(lse.cpu().numpy(), ref_lse, "draft_attn_window_fp8 lse")
 
 
+@pytest.mark.parametrize("W", [124, 316, 636, 1276, 2556])
+@pytest.mark.parametrize("n_q", [1, 4])
+def test_fp8_window_every_cluster_size(W, n_q):
+    """fp8 rings whose windows span 2, 5, 10, 20 and 40 tiles: the cluster window kernel with
+    1, 2, 4, 8 and 16 CTAs per unit, against the oracle on the dequantised cache."""
+    rng = np.random.default_rng(W + n_q)
+    B, Hq, Hkv, s = 2, 32, 4, 4
+    C = s + W
+    lens = [3 * C + 37, 2 * C + 5]
+    L = max(lens)
+    k_tok, v_tok = codes(rng, (B, L, Hkv, D)), codes(rng, (B, L, Hkv, D))
+    ring_k = dev8(np.full((B, Hkv, C, D), 0x7F, np.uint8))
+    ring_v = dev8(np.full((B, Hkv, C, D), 0x7F, np.uint8))
+    rlen = torch.zeros(B, dtype=torch.int64, device="cuda")
+    for b in range(B):
+        api.ring_kv_append_fp8(ring_k[b:b + 1], ring_v[b:b + 1], rlen[b:b + 1],
+                               dev8(k_tok[b:b + 1, :lens[b]]), dev8(v_tok[b:b + 1, :lens[b]]), s)
+    q = gen.normal_bf16(rng, (B, n_q, Hq, D))
+    ws = api.alloc_workspace(B, n_q, Hq, Hkv)
+    sc = 128 ** -0.5
+    out, lse = api.draft_attn_window_fp8(to_dev_bf16(q), ring_k, ring_v, rlen, s, W, sc, KS, VS, ws)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    k_lin = np.ascontiguousarray(k_tok.transpose(0, 2, 1, 3))
+    v_lin = np.ascontiguousarray(v_tok.transpose(0, 2, 1, 3))
+    ref, ref_lse = oracle.attention_kv8(q, k_lin, v_lin, np.array(lens), oracle.MODE_WINDOW, sc, KS, VS,
+                                        n_sink=s, window=W)
+    assert_attn_close(to_f64(out), ref, "draft_attn_window_fp8")
+    assert_lse_close(lse.cpu().numpy(), ref_lse, "draft_attn_window_fp8 lse")
+
+
 def test_fp8_equals_bf16_path_on_identical_values():
     """With unit scales, the fp8 call and the bf16 call on the same (exactly representable)
     numbers agree to within the two paths' rounding of the weights (fp16 vs bf16)."""
