@@ -151,16 +151,23 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.file.seek(0)
-        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.count(",") >= 6]
+        text = self.file.read()
         os.unlink(self.file.name)
-        if not rows:
-            return None
-        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].strip() == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        return parse_clock_samples(text)
+
+
+def parse_clock_samples(text: str):
+    """nvidia-smi CSV rows (ClockSampler.FIELDS, no header, no units) -> median SM clock under
+    load, the largest max clock, and every throttle reason seen Active; None without samples."""
+    rows = [r.split(",") for r in text.strip().splitlines() if r.count(",") >= 6]
+    if not rows:
+        return None
+    sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+    mx = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].strip() == "Active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
 # ----------------------------------------------------------------------------- GPU arm
