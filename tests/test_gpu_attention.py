@@ -225,11 +225,12 @@ def test_draft_window_matches_oracle(lens, Hq, Hkv, n_q, s, W, C):
 
 
 @pytest.mark.parametrize("W", [124, 316, 636, 1276, 2556])
-@pytest.mark.parametrize("n_q", [1, 4])
+@pytest.mark.parametrize("n_q", [1, 4, 8])
 def test_window_every_cluster_size(W, n_q):
     """Windows of 2, 5, 10, 20 and 40 tiles: the cluster window kernel runs with clusters of 1, 2,
     4, 8 and 16 CTAs per unit (the largest size that leaves each CTA at least two tiles), each
-    merging its partials through distributed shared memory; wrapped rings, ragged last tiles."""
+    merging its partials through distributed shared memory; 8, 32 and 64 rows per unit (its
+    three layouts); wrapped rings, ragged last tiles."""
     sc = 128 ** -0.5
     s = 4
     lens = [3 * (s + W) + 37, 2 * (s + W) + 5]

@@ -151,7 +151,7 @@ def test_ring_fp8_append_and_window_attention(L, n_q, s, W, C):
 
 
 @pytest.mark.parametrize("W", [124, 316, 636, 1276, 2556])
-@pytest.mark.parametrize("n_q", [1, 4])
+@pytest.mark.parametrize("n_q", [1, 4, 8])
 def test_fp8_window_every_cluster_size(W, n_q):
     """fp8 rings whose windows span 2, 5, 10, 20 and 40 tiles: the cluster window kernel with
     1, 2, 4, 8 and 16 CTAs per unit, against the oracle on the dequantised cache."""
